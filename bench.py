@@ -1,0 +1,373 @@
+"""Benchmark of the FFN-service MoE layer on B200: tokens/s per layer and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3_256] [--impl ours|reference]
+
+One step = one afd_ffn_forward over one micro-batch (router, top-k, dispatch, gate/up GEMM
+with SwiGLU, down GEMM, shared expert, combine).  Default workload: the DeepSeek-V3 shaped
+decode micro-batch (T=256, H=7168, E=256 + 1 shared, top-8, I=2048, bf16) on seeded
+synthetic inputs.  Its 22.6 GB of expert weights are far larger than the 126 MB L2, so no
+flush is needed between steps.  N > 1 runs one independent replica per GPU (the layer is
+not sharded: no collective on the data path); value = total tokens of all ranks / the
+slowest rank's time.  --impl reference times the fp64 CPU oracle on a bounded sample of the
+same workload instead (the reference arm).
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "MoE-FFN tokens/s/layer"
+
+
+# ----------------------------------------------------------------------------- accounting
+def touched_experts(counts, n_shared) -> int:
+    return int(np.count_nonzero(np.asarray(counts))) + n_shared
+
+
+def algorithmic(cfg, counts) -> dict:
+    """Per-forward algorithmic bytes and FLOPs (compulsory traffic only).
+
+    weights: every touched expert's W13 and W2 (+ e4m3 scales); activations: the hidden read,
+    the output write and the router weight read.  FLOPs: 6 H I (T k + S T) + 2 T H E.
+    gemm13: the gate/up GEMM alone -- touched W13 (+ scales), its dispatched input rows and its
+    SwiGLU output rows.
+    """
+    T, H, E, k, I, S = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.S
+    b = 1 if cfg.dtype == "fp8" else 2
+    n = touched_experts(counts, S)
+    w13 = n * (2 * I * H * b + (2 * I * 4 if b == 1 else 0))
+    w2 = n * (H * I * b + (H * 4 if b == 1 else 0))
+    act = T * H * 2 + T * H * 2 + E * H * 4
+    rows = T * k + S * T
+    gemm13 = w13 + rows * H * b + rows * I * (4 if b == 1 else 2)
+    flops = 6 * H * I * (T * k + S * T) + 2 * T * H * E
+    return {"weight_bytes": w13 + w2, "act_bytes": act, "flops": flops, "gemm13_bytes": gemm13,
+            "gemm13_flops": 4 * H * I * rows, "touched_experts": n}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if self.proc is None or self.f is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.flush()
+        with open(self.f.name) as fh:
+            rows = [r.split(",") for r in fh.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        busy = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def build_inputs(cfg, device):
+    hidden = synth.gen_hidden(cfg)
+    Wr, bias = synth.gen_router(cfg)
+    ex = synth.gen_experts(cfg)
+    dev = {k: v.to(device) for k, v in ex.items()}
+    dev["router_w"] = Wr.to(device)
+    if bias is not None:
+        dev["router_bias"] = bias.to(device)
+    return hidden, Wr, bias, ex, dev
+
+
+def cpu_baseline(cfg, hidden, Wr, bias, ex, budget_s=15.0) -> dict:
+    """The fp64 oracle, as it stands, on the first few tokens of the same micro-batch."""
+    from oracle import moe
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        blas = None
+    cores = len(os.sched_getaffinity(0))
+    fn = lambda e: {kk: v[e] for kk, v in ex.items()}  # noqa: E731
+    n, spent, done = 1, 0.0, 0
+    while True:
+        t0 = time.perf_counter()
+        moe.forward(hidden[:n], Wr, bias, fn, cfg.E, cfg.k, cfg.S, fp8=cfg.dtype == "fp8")
+        dt = time.perf_counter() - t0
+        spent, done = dt, n
+        if dt > budget_s / 3 or n >= cfg.T:
+            break
+        n = min(cfg.T, n * 4)
+    return {"value": done / spent, "unit": "tokens/s", "cores": blas or cores, "host_cores": cores,
+            "kind": "oracle",
+            "sample": f"first {done} of {cfg.T} tokens of the {cfg.name} micro-batch, full fp64 layer "
+                      f"(routing, {cfg.k} experts + {cfg.S} shared per token), {spent:.1f} s"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import ffn_side_expert_b200 as afd
+    cfg = synth.CONFIGS[args.config]
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    hidden, Wr, bias, ex, dev = build_inputs(cfg, device)
+    layer = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S,
+                       fp8=cfg.dtype == "fp8", weights=dev)
+    h = hidden.to(device)
+    out = torch.empty_like(h)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        layer.forward(h, out)
+    torch.cuda.synchronize()
+    st = layer.get_error()
+    if st != afd.AFD_OK:
+        raise afd.AfdError(st, "warm-up")
+
+    # routing counts of this micro-batch (for the touched-expert byte count)
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=device)
+    wts = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=device)
+    layer.route(h, cfg.T, idx, wts)
+    counts = np.bincount(idx.cpu().numpy().ravel(), minlength=cfg.E)
+    acct = algorithmic(cfg, counts)
+
+    # per-step stage events: AFD_FFN_NUM_STAGES + 1 per step, recorded on the launch stream
+    nev = afd.AFD_FFN_NUM_STAGES + 1
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            layer.set_stage_events(ev[i])
+            layer.forward(h, out)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    layer.set_stage_events(None)
+    ms = t_start.elapsed_time(t_end) / args.steps
+    st = layer.get_error()
+    if st != afd.AFD_OK:
+        raise afd.AfdError(st, "timed region")
+    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(nev - 1)]
+                         for i in range(args.steps)]).mean(axis=0)
+
+    # end to end: host buffers through the C ABI, copies inside the timed region
+    hin = hidden.clone().pin_memory()
+    hout = torch.empty_like(hin).pin_memory()
+    layer.forward_host(hin, hout)
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        layer.forward_host(hin, hout)
+    e2e_s = (time.perf_counter() - t0) / args.steps
+
+    ms_max = allreduce_max(ms, world)
+    e2e_max = allreduce_max(e2e_s, world)
+    res = {"ms": ms_max, "e2e_s": e2e_max, "stage_ms": stage_ms, "acct": acct, "cfg": cfg,
+           "clocks": clk.summary(), "bytes_io": hidden.numel() * 2}
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu"] = cpu_baseline(cfg, hidden, Wr, bias, ex)
+    layer.close()
+    return res
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def report_ours(args, world, r) -> dict:
+    import ffn_side_expert_b200 as afd
+    cfg, acct = r["cfg"], r["acct"]
+    peaks, kind = load_peaks()
+    ms = r["ms"]
+    value = world * cfg.T / (ms / 1e3)
+    stage = dict(zip(afd.STAGE_NAMES, [float(x) for x in r["stage_ms"]]))
+    g13_ms = stage["gemm_gate_up"]
+    hbm = peaks["hbm_gbs"]
+    achieved = acct["gemm13_bytes"] / (g13_ms / 1e3) / 1e9
+    t_hbm = (acct["weight_bytes"] + acct["act_bytes"]) / (hbm * 1e9)
+    tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.dtype == "fp8" else 1.0)
+    t_tc = acct["flops"] / (tc_peak * 1e12)
+    t_roof = max(t_hbm, t_tc)
+    launches = 9 if cfg.dtype == "fp8" else 8
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if cfg.dtype == "fp8" else "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+                   "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (expert weights 22.6 GB >> 126 MB)"},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm gate/up + SwiGLU",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "peak_source": f"{kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": acct["gemm13_bytes"],
+                     "avg_launch_ms": round(g13_ms, 4)},
+        "path_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
+                          "t_tensor_ms": round(t_tc * 1e3, 4), "frac": round(t_roof * 1e3 / ms, 4),
+                          "weight_bytes": acct["weight_bytes"], "act_bytes": acct["act_bytes"],
+                          "flops": acct["flops"], "touched_experts": acct["touched_experts"],
+                          "peaks": f"{kind}: hbm {hbm} GB/s, tensor {tc_peak} TFLOP/s"},
+        "stage_ms": {k: round(v, 4) for k, v in stage.items()},
+        "e2e": {"value": round(world * cfg.T / r["e2e_s"], 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["bytes_io"], "d2h_bytes_per_step": r["bytes_io"]},
+        "gpu_launches": launches * args.steps,
+        "clocks": r["clocks"],
+        "cpu_baseline": r.get("cpu"),
+    }
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle timed on the host, a bounded token sample per step."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import moe
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    hidden = synth.gen_hidden(cfg)
+    Wr, bias = synth.gen_router(cfg)
+    n = max(1, int(args.ref_tokens))
+    plan = [[(i * n + j) % cfg.T for j in range(n)] for i in range(args.warmup + args.steps)]
+    # the experts the sampled tokens visit are drawn before any timing
+    _, idx, _ = moe.route(hidden[sorted({t for p in plan for t in p})], Wr, bias, cfg.k)
+    need = sorted(set(np.unique(idx).tolist()) | set(range(cfg.E, cfg.E + cfg.S)))
+    with ThreadPoolExecutor(max(1, min(16, len(os.sched_getaffinity(0))))) as ex:
+        cache = dict(zip(need, ex.map(lambda e: synth.gen_expert(cfg, e), need)))
+    steps = []
+    for i, tok in enumerate(plan):
+        t0 = time.perf_counter()
+        moe.forward(hidden, Wr, bias, cache.__getitem__, cfg.E, cfg.k, cfg.S, fp8=cfg.dtype == "fp8",
+                    tokens=tok)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            steps.append(dt)
+    per_tok = sum(steps) / (n * len(steps))
+    value = 1.0 / per_tok
+    cores = len(os.sched_getaffinity(0))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * per_tok * cfg.T, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+                   "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} token(s) of the {cfg.name} micro-batch per step, full fp64 layer "
+                                   f"(expert weights drawn before timing); ms_per_step scaled to T={cfg.T}"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="dsv3_256", choices=list(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=1, help="reference arm: tokens per step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(report_ours(args, world, r)), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,241 @@
+"""Python binding of libafd_ffn.so, the FFN-service MoE layer of Attention-FFN Disaggregation
+on one B200.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.  The
+functions below carry the C names of include/afd_ffn.h and return its status codes; the
+``AfdFfn`` class wraps a handle, keeps the borrowed weight tensors alive, and raises
+``AfdError`` on a non-zero status.  torch is used only for device memory and streams.
+
+Importing fails (ImportError) when the library has not been built:
+``python ffn_side_expert_b200/build.py``.  There is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libafd_ffn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "afd_ffn.h")
+
+AFD_OK = 0
+AFD_ERR_INVALID_ARG = -1
+AFD_ERR_UNSUPPORTED = -2
+AFD_ERR_T_TOO_LARGE = -3
+AFD_ERR_CUDA = -4
+AFD_ERR_DEVICE_FLAG = -5
+AFD_ERR_DEVICE_TIMEOUT = -6
+AFD_ERR_NO_DEVICE = -7
+AFD_DT_BF16 = 0
+AFD_DT_FP8_E4M3 = 1
+AFD_FFN_NUM_STAGES = 9
+STAGE_NAMES = ("router_logits", "router_topk", "dispatch_order", "gather_rows", "gemm_schedule",
+               "gemm_gate_up", "quantize_act", "gemm_down", "combine")
+
+
+class afd_ffn_cfg(ctypes.Structure):
+    _fields_ = [("T_max", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("weight_dtype", ctypes.c_int32), ("act_dtype", ctypes.c_int32),
+                ("has_router_bias", ctypes.c_int32)]
+
+
+class afd_ffn_weights(ctypes.Structure):
+    _fields_ = [("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("w13_scale", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_SIGNATURES = {
+    "afd_ffn_create": (ctypes.c_int, [ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(afd_ffn_weights),
+                                      ctypes.POINTER(ctypes.c_void_p)]),
+    "afd_ffn_destroy": (None, [_P]),
+    "afd_ffn_route": (ctypes.c_int, [_P, _P, _I, _P, _P, _P]),
+    "afd_ffn_permute": (ctypes.c_int, [_P, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "afd_ffn_expert_gemm": (ctypes.c_int, [_P, _P, _I, _P, _P, _P]),
+    "afd_ffn_combine": (ctypes.c_int, [_P, _P, _P, _I, _P, _P]),
+    "afd_ffn_forward": (ctypes.c_int, [_P, _P, _I, _P, _P]),
+    "afd_ffn_forward_host": (ctypes.c_int, [_P, _P, _I, _P, _P]),
+    "afd_ffn_set_stage_events": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
+    "afd_ffn_get_error": (ctypes.c_int, [_P]),
+    "afd_ffn_last_cuda_error": (ctypes.c_int, [_P]),
+    "afd_ffn_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python ffn_side_expert_b200/build.py` "
+                          "(the layer has no CPU or library fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def declared_functions(header: str = HEADER_PATH) -> list:
+    """Names of the entry points declared in include/afd_ffn.h."""
+    with open(header) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(afd_ffn_\w+)\s*\(", text)))
+
+
+class AfdError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {afd_ffn_strerror(status)} ({status})")
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ------------------------------------------------------------------ C entry points
+def afd_ffn_strerror(status: int) -> str:
+    return _lib.afd_ffn_strerror(status).decode()
+
+
+def afd_ffn_create(cfg: afd_ffn_cfg, weights: afd_ffn_weights):
+    """Returns (status, handle or None)."""
+    h = ctypes.c_void_p()
+    st = _lib.afd_ffn_create(ctypes.byref(cfg) if cfg is not None else None,
+                             ctypes.byref(weights) if weights is not None else None, ctypes.byref(h))
+    return st, (h.value if st == AFD_OK else None)
+
+
+def afd_ffn_destroy(h) -> None:
+    _lib.afd_ffn_destroy(h)
+
+
+def afd_ffn_route(h, hidden, T, topk_idx, topk_w, stream=None) -> int:
+    return _lib.afd_ffn_route(h, _ptr(hidden), T, _ptr(topk_idx), _ptr(topk_w), _stream(stream))
+
+
+def afd_ffn_permute(h, hidden, topk_idx, T, counts, offsets, pos, src, stream=None) -> int:
+    return _lib.afd_ffn_permute(h, _ptr(hidden), _ptr(topk_idx), T, _ptr(counts), _ptr(offsets), _ptr(pos),
+                                _ptr(src), _stream(stream))
+
+
+def afd_ffn_expert_gemm(h, offsets, T, Y=None, Ys=None, stream=None) -> int:
+    return _lib.afd_ffn_expert_gemm(h, _ptr(offsets), T, _ptr(Y), _ptr(Ys), _stream(stream))
+
+
+def afd_ffn_combine(h, topk_w, pos, T, out, stream=None) -> int:
+    return _lib.afd_ffn_combine(h, _ptr(topk_w), _ptr(pos), T, _ptr(out), _stream(stream))
+
+
+def afd_ffn_forward(h, hidden, T, out, stream=None) -> int:
+    return _lib.afd_ffn_forward(h, _ptr(hidden), T, _ptr(out), _stream(stream))
+
+
+def afd_ffn_forward_host(h, hidden_host, T, out_host, stream=None) -> int:
+    return _lib.afd_ffn_forward_host(h, _ptr(hidden_host), T, _ptr(out_host), _stream(stream))
+
+
+def afd_ffn_set_stage_events(h, events) -> int:
+    """events: sequence of torch.cuda.Event (AFD_FFN_NUM_STAGES + 1 of them) or None."""
+    if not events:
+        return _lib.afd_ffn_set_stage_events(h, None, 0)
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    return _lib.afd_ffn_set_stage_events(h, arr, len(events))
+
+
+def afd_ffn_get_error(h) -> int:
+    return _lib.afd_ffn_get_error(h)
+
+
+def afd_ffn_last_cuda_error(h) -> int:
+    return _lib.afd_ffn_last_cuda_error(h)
+
+
+# ------------------------------------------------------------------ convenience wrapper
+class AfdFfn:
+    """A handle on the current CUDA device.
+
+    weights: dict with device tensors router_w [E,H] fp32, optional router_bias [E] fp32,
+    w13 [E+S,2I,H] and w2 [E+S,H,I] (bf16 or float8_e4m3fn), and for e4m3 w13_scale [E+S,2I],
+    w2_scale [E+S,H] fp32.  The tensors are referenced for the handle's lifetime.
+    """
+
+    def __init__(self, *, T_max, H, E, k, I, n_shared, fp8, weights):
+        dt = AFD_DT_FP8_E4M3 if fp8 else AFD_DT_BF16
+        self.cfg = afd_ffn_cfg(T_max, H, E, k, I, n_shared, dt, dt,
+                               1 if weights.get("router_bias") is not None else 0)
+        self._keep = dict(weights)
+        w = afd_ffn_weights(_ptr(weights["router_w"]), _ptr(weights.get("router_bias")),
+                            _ptr(weights["w13"]), _ptr(weights["w2"]),
+                            _ptr(weights.get("w13_scale")), _ptr(weights.get("w2_scale")))
+        st, self.h = afd_ffn_create(self.cfg, w)
+        if st != AFD_OK:
+            raise AfdError(st, "afd_ffn_create")
+        self._events = None
+
+    def close(self):
+        if getattr(self, "h", None):
+            afd_ffn_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st, what):
+        if st != AFD_OK:
+            raise AfdError(st, what)
+
+    def route(self, hidden, T, topk_idx, topk_w, stream=None):
+        self._check(afd_ffn_route(self.h, hidden, T, topk_idx, topk_w, stream), "afd_ffn_route")
+
+    def permute(self, hidden, topk_idx, T, counts, offsets, pos, src, stream=None):
+        self._check(afd_ffn_permute(self.h, hidden, topk_idx, T, counts, offsets, pos, src, stream),
+                    "afd_ffn_permute")
+
+    def expert_gemm(self, offsets, T, Y=None, Ys=None, stream=None):
+        self._check(afd_ffn_expert_gemm(self.h, offsets, T, Y, Ys, stream), "afd_ffn_expert_gemm")
+
+    def combine(self, topk_w, pos, T, out, stream=None):
+        self._check(afd_ffn_combine(self.h, topk_w, pos, T, out, stream), "afd_ffn_combine")
+
+    def forward(self, hidden, out, T=None, stream=None):
+        T = hidden.shape[0] if T is None else T
+        self._check(afd_ffn_forward(self.h, hidden, T, out, stream), "afd_ffn_forward")
+
+    def forward_host(self, hidden_host, out_host, T=None, stream=None):
+        T = hidden_host.shape[0] if T is None else T
+        self._check(afd_ffn_forward_host(self.h, hidden_host, T, out_host, stream), "afd_ffn_forward_host")
+
+    def set_stage_events(self, events):
+        self._events = events          # keep the events alive while the library records them
+        self._check(afd_ffn_set_stage_events(self.h, events), "afd_ffn_set_stage_events")
+
+    def get_error(self) -> int:
+        return afd_ffn_get_error(self.h)
+
+
+__all__ = [n for n in list(globals()) if n.startswith(("afd_ffn", "AFD_", "Afd"))] + [
+    "declared_functions", "LIB_PATH", "STAGE_NAMES"]

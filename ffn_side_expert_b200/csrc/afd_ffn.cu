@@ -1,0 +1,523 @@
+// afd_ffn.cu -- host side of libafd_ffn.so: argument checks, workspace, TMA descriptors and
+// the launch sequence of the FFN-service MoE layer.  The declarations, conventions and
+// readings are documented in include/afd_ffn.h.
+//
+// Launch sequence of afd_ffn_forward (one stream, no host synchronisation):
+//   router_logits -> router_topk -> dispatch_order -> gather_rows (W8A8: + quantise) ->
+//   build_schedule -> grouped_gemm<gate/up> -> (W8A8: quantize_act) -> grouped_gemm<down>
+//   -> combine
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "afd_ffn.h"
+#include "combine.cuh"
+#include "dispatch.cuh"
+#include "gemm.cuh"
+#include "router.cuh"
+
+using namespace afd;
+
+namespace {
+
+// Two tile shapes of the grouped GEMM: "narrow" for decode micro-batches (a few rows per
+// expert: N <= 32, a deep ring of small stages, double-buffered TMEM) and "wide" for large
+// micro-batches (N <= 256, the widest MMA; three 64 KB stages).
+constexpr int kNarrowBN = 32, kNarrowStages = 6;
+constexpr int kWideBN = 256, kWideStages = 3;
+
+thread_local int g_create_cuda_error = 0;
+
+}  // namespace
+
+struct afd_ffn_handle {
+  afd_ffn_cfg cfg;
+  afd_ffn_weights w;
+  int device = 0;
+  int num_sms = 0;
+  bool fp8 = false;
+  int G = 0;       // E + n_shared
+  int R_max = 0;   // rows of the dispatched-row buffers: T_max * (k + 1)
+  size_t part_floats = 0;
+
+  void* ws = nullptr;
+  float* part = nullptr;
+  int32_t* idx = nullptr;
+  float* wts = nullptr;
+  int32_t* counts = nullptr;
+  int32_t* offsets = nullptr;
+  int32_t* pos = nullptr;
+  int32_t* src = nullptr;
+  int32_t* grp_rows = nullptr;
+  int32_t* grp_base = nullptr;
+  int32_t* ub1 = nullptr;
+  int32_t* ub2 = nullptr;
+  uint8_t* xp = nullptr;     // dispatched rows [R_max][H] bf16 / e4m3
+  float* xscale = nullptr;   // [R_max]
+  void* act = nullptr;       // [R_max][I] bf16 (or fp32 in W8A8)
+  uint8_t* actq = nullptr;   // W8A8: [R_max][I] e4m3
+  float* ascale = nullptr;   // W8A8: [R_max]
+  float* Y = nullptr;        // [R_max][H] fp32
+  int* err = nullptr;        // device error word
+  void* hin = nullptr;       // [T_max][H] bf16 staging for afd_ffn_forward_host
+  void* hout = nullptr;
+
+  CUtensorMap tm_w13, tm_w2, tm_xp, tm_act;
+  cudaStream_t last_stream = nullptr;
+  int last_cuda_error = 0;
+  cudaEvent_t events[AFD_FFN_NUM_STAGES + 1];
+  int n_events = 0;
+};
+
+namespace {
+
+int cuda_fail(afd_ffn_handle* h, cudaError_t e) {
+  if (h) h->last_cuda_error = static_cast<int>(e); else g_create_cuda_error = static_cast<int>(e);
+  return AFD_ERR_CUDA;
+}
+
+#define AFD_CUDA(h, call)                                  \
+  do {                                                     \
+    cudaError_t e_ = (call);                               \
+    if (e_ != cudaSuccess) return cuda_fail((h), e_);      \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void router_split(int T, int H, int E, int sms, int* nsplit, int* per) {
+  const int tiles = ((T + kRtTok - 1) / kRtTok) * ((E + kRtExp - 1) / kRtExp);
+  const int kt = H / kRtK;
+  int want = std::max(1, (2 * sms + tiles - 1) / std::max(tiles, 1));
+  want = std::min(want, std::min(32, kt));
+  *per = (kt + want - 1) / want;
+  *nsplit = (kt + *per - 1) / *per;
+}
+
+bool use_narrow(const afd_ffn_handle* h, int T) {
+  return static_cast<long long>(T) * h->cfg.k <= 32LL * h->cfg.E;
+}
+
+int check_device(afd_ffn_handle* h) {
+  int dev = -1;
+  AFD_CUDA(h, cudaGetDevice(&dev));
+  if (dev != h->device) return AFD_ERR_INVALID_ARG;
+  return AFD_OK;
+}
+
+int check_T(const afd_ffn_handle* h, int32_t T) {
+  if (T < 0) return AFD_ERR_INVALID_ARG;
+  if (T > h->cfg.T_max) return AFD_ERR_T_TOO_LARGE;
+  return AFD_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D K-major tensor [rows][inner] of 1- or 2-byte elements; box = (128 bytes) x box_rows,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner, uint64_t rows,
+               uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  const uint32_t esz = byte_elems ? 1 : 2;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {128u / esz, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, byte_elems ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, bool FP8, int MODE>
+cudaError_t set_gemm_attr() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8, MODE>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, STAGES>());
+}
+
+template <bool FP8>
+cudaError_t set_all_gemm_attrs() {
+  cudaError_t e;
+  if ((e = set_gemm_attr<kNarrowBN, kNarrowStages, FP8, 0>()) != cudaSuccess) return e;
+  if ((e = set_gemm_attr<kNarrowBN, kNarrowStages, FP8, 1>()) != cudaSuccess) return e;
+  if ((e = set_gemm_attr<kWideBN, kWideStages, FP8, 0>()) != cudaSuccess) return e;
+  return set_gemm_attr<kWideBN, kWideStages, FP8, 1>();
+}
+
+template <int BN, int STAGES, bool FP8, int MODE>
+void launch_gemm(const afd_ffn_handle* h, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args,
+                 cudaStream_t s) {
+  grouped_gemm_kernel<BN, STAGES, FP8, MODE>
+      <<<h->num_sms, 192, gemm_smem_bytes<BN, STAGES>(), s>>>(a, b, args);
+}
+
+void record(afd_ffn_handle* h, int stage, cudaStream_t s) {
+  if (h->n_events > stage) cudaEventRecord(h->events[stage], s);
+}
+
+// ------------------------------------------------------------------ stages
+int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float* w, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  int nsplit = 1, per = 1;
+  router_split(T, c.H, c.E, h->num_sms, &nsplit, &per);
+  record(h, 0, s);
+  dim3 grid((c.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
+  router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, h->part, T,
+                                            c.H, c.E, per);
+  record(h, 1, s);
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, nsplit, c.has_router_bias ? h->w.router_bias : nullptr, T,
+                                                 c.E, c.k, idx, w);
+  AFD_CUDA(h, cudaGetLastError());
+  return AFD_OK;
+}
+
+int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T, int32_t* counts, int32_t* offsets,
+                int32_t* pos, int32_t* src, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  record(h, 2, s);
+  dispatch_order_kernel<<<1, kDispatchThreads, 0, s>>>(idx, T, c.k, c.E, counts, offsets, pos, src, h->err);
+  record(h, 3, s);
+  if (h->fp8)
+    gather_rows_kernel<true><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), pos, T, c.k, c.H, T * c.k,
+                                               c.n_shared, T * c.k, h->xp, h->xscale, h->err);
+  else
+    gather_rows_kernel<false><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), pos, T, c.k, c.H,
+                                                T * c.k, c.n_shared, T * c.k, h->xp, h->xscale, h->err);
+  AFD_CUDA(h, cudaGetLastError());
+  return AFD_OK;
+}
+
+template <int BN, int STAGES, bool FP8>
+void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  const int R = T * c.k + T;
+  GemmArgs g1{};
+  g1.grp_rows = h->grp_rows;
+  g1.grp_base = h->grp_base;
+  g1.unit_base = h->ub1;
+  g1.G = h->G;
+  g1.K = c.H;
+  g1.a_rows = 2 * c.I;
+  g1.mt_stride = 128;
+  g1.second_off = c.I;
+  g1.out = h->act;
+  g1.out_ld = c.I;
+  g1.a_scale = h->w.w13_scale;
+  g1.b_scale = h->xscale;
+  g1.err = h->err;
+  record(h, 5, s);
+  launch_gemm<BN, STAGES, FP8, 0>(h, h->tm_w13, h->tm_xp, g1, s);
+  record(h, 6, s);
+  if (FP8) quantize_act_kernel<<<R, 256, 0, s>>>(static_cast<const float*>(h->act), c.I, h->actq, h->ascale);
+  GemmArgs g2 = g1;
+  g2.unit_base = h->ub2;
+  g2.K = c.I;
+  g2.a_rows = c.H;
+  g2.mt_stride = 256;
+  g2.second_off = 128;
+  g2.out = h->Y;
+  g2.out_ld = c.H;
+  g2.a_scale = h->w.w2_scale;
+  g2.b_scale = h->ascale;
+  record(h, 7, s);
+  launch_gemm<BN, STAGES, FP8, 1>(h, h->tm_w2, h->tm_act, g2, s);
+}
+
+int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  const bool narrow = use_narrow(h, T);
+  const int bn = narrow ? kNarrowBN : kWideBN;
+  record(h, 4, s);
+  build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn, c.I / 128, c.H / 256, h->grp_rows,
+                                          h->grp_base, h->ub1, h->ub2, h->err);
+  if (h->fp8) {
+    if (narrow) run_gemms<kNarrowBN, kNarrowStages, true>(h, T, s);
+    else run_gemms<kWideBN, kWideStages, true>(h, T, s);
+  } else {
+    if (narrow) run_gemms<kNarrowBN, kNarrowStages, false>(h, T, s);
+    else run_gemms<kWideBN, kWideStages, false>(h, T, s);
+  }
+  AFD_CUDA(h, cudaGetLastError());
+  return AFD_OK;
+}
+
+int run_combine(afd_ffn_handle* h, const float* w, const int32_t* pos, int T, void* out, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  record(h, 8, s);
+  combine_kernel<<<T, 256, 0, s>>>(h->Y, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
+                                   static_cast<__nv_bfloat16*>(out), h->err);
+  record(h, 9, s);
+  AFD_CUDA(h, cudaGetLastError());
+  return AFD_OK;
+}
+
+int validate_cfg(const afd_ffn_cfg* c) {
+  if (c->T_max < 1 || c->H < 1 || c->E < 1 || c->k < 1 || c->I < 1) return AFD_ERR_INVALID_ARG;
+  if (c->n_shared != 0 && c->n_shared != 1) return AFD_ERR_INVALID_ARG;
+  if (c->has_router_bias != 0 && c->has_router_bias != 1) return AFD_ERR_INVALID_ARG;
+  if (c->weight_dtype != AFD_DT_BF16 && c->weight_dtype != AFD_DT_FP8_E4M3) return AFD_ERR_INVALID_ARG;
+  if (c->act_dtype != c->weight_dtype) return AFD_ERR_UNSUPPORTED;
+  if (c->k > c->E) return AFD_ERR_INVALID_ARG;
+  if (c->E > kMaxExperts || c->k > 32) return AFD_ERR_UNSUPPORTED;
+  if (c->H % 256 != 0 || c->I % 128 != 0) return AFD_ERR_UNSUPPORTED;
+  // dispatched rows and per-row offsets must fit int32; TMA row coordinates too
+  const long long rows = static_cast<long long>(c->T_max) * (c->k + 1);
+  if (rows > (1LL << 30) || static_cast<long long>(c->E + 1) * 2 * c->I > (1LL << 30) ||
+      static_cast<long long>(c->E + 1) * c->H > (1LL << 30))
+    return AFD_ERR_UNSUPPORTED;
+  return AFD_OK;
+}
+
+int validate_weights(const afd_ffn_cfg* c, const afd_ffn_weights* w) {
+  if (!w->router_w || !w->w13 || !w->w2) return AFD_ERR_INVALID_ARG;
+  if (c->has_router_bias && !w->router_bias) return AFD_ERR_INVALID_ARG;
+  if (!c->has_router_bias && w->router_bias) return AFD_ERR_INVALID_ARG;
+  const bool fp8 = c->weight_dtype == AFD_DT_FP8_E4M3;
+  if (fp8 && (!w->w13_scale || !w->w2_scale)) return AFD_ERR_INVALID_ARG;
+  if (!fp8 && (w->w13_scale || w->w2_scale)) return AFD_ERR_INVALID_ARG;
+  if (!aligned16(w->router_w) || !aligned16(w->w13) || !aligned16(w->w2)) return AFD_ERR_INVALID_ARG;
+  return AFD_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* afd_ffn_strerror(int status) {
+  switch (status) {
+    case AFD_OK: return "ok";
+    case AFD_ERR_INVALID_ARG: return "invalid argument";
+    case AFD_ERR_UNSUPPORTED: return "configuration not supported";
+    case AFD_ERR_T_TOO_LARGE: return "T exceeds the handle's T_max";
+    case AFD_ERR_CUDA: return "CUDA call failed";
+    case AFD_ERR_DEVICE_FLAG: return "device skipped invalid data (expert index or position)";
+    case AFD_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
+    case AFD_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+    default: return "unknown status";
+  }
+}
+
+int afd_ffn_last_cuda_error(const afd_ffn_handle* h) { return h ? h->last_cuda_error : g_create_cuda_error; }
+
+int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_ffn_handle** out) {
+  if (!out) return AFD_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !weights) return AFD_ERR_INVALID_ARG;
+  int st = validate_cfg(cfg);
+  if (st != AFD_OK) return st;
+  if ((st = validate_weights(cfg, weights)) != AFD_OK) return st;
+  g_create_cuda_error = 0;
+
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) { g_create_cuda_error = e; return AFD_ERR_NO_DEVICE; }
+  int major = 0, minor = 0, sms = 0;
+  AFD_CUDA(nullptr, cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  AFD_CUDA(nullptr, cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  AFD_CUDA(nullptr, cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  if (major != 10 || minor != 0) return AFD_ERR_NO_DEVICE;
+  if (!get_encode()) return AFD_ERR_NO_DEVICE;
+
+  afd_ffn_handle* h = new (std::nothrow) afd_ffn_handle();
+  if (!h) return AFD_ERR_INVALID_ARG;
+  h->cfg = *cfg;
+  h->w = *weights;
+  h->device = dev;
+  h->num_sms = sms;
+  h->fp8 = cfg->weight_dtype == AFD_DT_FP8_E4M3;
+  h->G = cfg->E + cfg->n_shared;
+  h->R_max = cfg->T_max * (cfg->k + 1);
+
+  const afd_ffn_cfg& c = h->cfg;
+  size_t part = 0;
+  for (int T = 1; T <= c.T_max; ++T) {
+    int ns, per;
+    router_split(T, c.H, c.E, sms, &ns, &per);
+    part = std::max(part, static_cast<size_t>(ns) * T * c.E);
+  }
+  h->part_floats = part;
+
+  // one allocation, 256-byte aligned pieces
+  const size_t R = h->R_max, Tm = c.T_max, wb = h->fp8 ? 1 : 2;
+  struct Piece { void** p; size_t bytes; };
+  void* act_p = nullptr;
+  Piece pieces[] = {
+      {reinterpret_cast<void**>(&h->part), part * 4},
+      {reinterpret_cast<void**>(&h->idx), Tm * c.k * 4},
+      {reinterpret_cast<void**>(&h->wts), Tm * c.k * 4},
+      {reinterpret_cast<void**>(&h->counts), static_cast<size_t>(c.E) * 4},
+      {reinterpret_cast<void**>(&h->offsets), static_cast<size_t>(c.E + 1) * 4},
+      {reinterpret_cast<void**>(&h->pos), Tm * c.k * 4},
+      {reinterpret_cast<void**>(&h->src), Tm * c.k * 4},
+      {reinterpret_cast<void**>(&h->grp_rows), static_cast<size_t>(h->G) * 4},
+      {reinterpret_cast<void**>(&h->grp_base), static_cast<size_t>(h->G) * 4},
+      {reinterpret_cast<void**>(&h->ub1), static_cast<size_t>(h->G + 1) * 4},
+      {reinterpret_cast<void**>(&h->ub2), static_cast<size_t>(h->G + 1) * 4},
+      {reinterpret_cast<void**>(&h->xp), R * c.H * wb},
+      {reinterpret_cast<void**>(&h->xscale), R * 4},
+      {&act_p, R * c.I * (h->fp8 ? 4 : 2)},
+      {reinterpret_cast<void**>(&h->actq), h->fp8 ? R * c.I : 0},
+      {reinterpret_cast<void**>(&h->ascale), R * 4},
+      {reinterpret_cast<void**>(&h->Y), R * c.H * 4},
+      {reinterpret_cast<void**>(&h->err), 256},
+      {&h->hin, Tm * c.H * 2},
+      {&h->hout, Tm * c.H * 2},
+  };
+  size_t total = 0;
+  for (auto& p : pieces) total += (p.bytes + 255) & ~size_t(255);
+  e = cudaMalloc(&h->ws, total);
+  if (e != cudaSuccess) { delete h; return cuda_fail(nullptr, e); }
+  e = cudaMemset(h->ws, 0, total);
+  if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  size_t off = 0;
+  for (auto& p : pieces) {
+    *p.p = p.bytes ? static_cast<uint8_t*>(h->ws) + off : nullptr;
+    off += (p.bytes + 255) & ~size_t(255);
+  }
+  h->act = act_p;
+
+  const uint64_t G = h->G;
+  bool ok = encode_2d(&h->tm_w13, weights->w13, h->fp8, c.H, G * 2 * c.I, 128) &&
+            encode_2d(&h->tm_w2, weights->w2, h->fp8, c.I, G * c.H, 128) &&
+            encode_2d(&h->tm_xp, h->xp, h->fp8, c.H, R, 16) &&
+            encode_2d(&h->tm_act, h->fp8 ? static_cast<const void*>(h->actq) : h->act, h->fp8, c.I, R, 16);
+  if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
+  e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
+  if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  *out = h;
+  return AFD_OK;
+}
+
+void afd_ffn_destroy(afd_ffn_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  cudaFree(h->ws);
+  delete h;
+}
+
+int afd_ffn_route(afd_ffn_handle* h, const void* hidden, int32_t T, int32_t* topk_idx, float* topk_w, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (T == 0) return AFD_OK;
+  if (!hidden || !topk_idx || !topk_w || !aligned16(hidden)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  return run_route(h, hidden, T, topk_idx, topk_w, s);
+}
+
+int afd_ffn_permute(afd_ffn_handle* h, const void* hidden, const int32_t* topk_idx, int32_t T, int32_t* counts,
+                    int32_t* offsets, int32_t* pos, int32_t* src, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (!hidden || !topk_idx || !counts || !offsets || !pos || !src || !aligned16(hidden)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (T == 0) {  // no pairs: zero counts and offsets
+    AFD_CUDA(h, cudaMemsetAsync(counts, 0, sizeof(int32_t) * h->cfg.E, s));
+    AFD_CUDA(h, cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (h->cfg.E + 1), s));
+    return AFD_OK;
+  }
+  return run_permute(h, hidden, topk_idx, T, counts, offsets, pos, src, s);
+}
+
+int afd_ffn_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int32_t T, float* Y, float* Ys, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (!offsets) return AFD_ERR_INVALID_ARG;
+  if (Ys && h->cfg.n_shared == 0) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  if (T == 0) return AFD_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if ((st = run_expert_gemm(h, offsets, T, s)) != AFD_OK) return st;
+  const size_t H = h->cfg.H, rk = static_cast<size_t>(T) * h->cfg.k;
+  if (Y) AFD_CUDA(h, cudaMemcpyAsync(Y, h->Y, rk * H * 4, cudaMemcpyDeviceToDevice, s));
+  if (Ys) AFD_CUDA(h, cudaMemcpyAsync(Ys, h->Y + rk * H, static_cast<size_t>(T) * H * 4, cudaMemcpyDeviceToDevice, s));
+  return AFD_OK;
+}
+
+int afd_ffn_combine(afd_ffn_handle* h, const float* topk_w, const int32_t* pos, int32_t T, void* out, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (T == 0) return AFD_OK;
+  if (!topk_w || !pos || !out || !aligned16(out)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  return run_combine(h, topk_w, pos, T, out, s);
+}
+
+int afd_ffn_forward(afd_ffn_handle* h, const void* hidden, int32_t T, void* out, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (T == 0) return AFD_OK;
+  if (!hidden || !out || !aligned16(hidden) || !aligned16(out)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if ((st = run_route(h, hidden, T, h->idx, h->wts, s)) != AFD_OK) return st;
+  if ((st = run_permute(h, hidden, h->idx, T, h->counts, h->offsets, h->pos, h->src, s)) != AFD_OK) return st;
+  if ((st = run_expert_gemm(h, h->offsets, T, s)) != AFD_OK) return st;
+  return run_combine(h, h->wts, h->pos, T, out, s);
+}
+
+int afd_ffn_forward_host(afd_ffn_handle* h, const void* hidden_host, int32_t T, void* out_host, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (T == 0) return AFD_OK;
+  if (!hidden_host || !out_host) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * h->cfg.H * 2;
+  AFD_CUDA(h, cudaMemcpyAsync(h->hin, hidden_host, bytes, cudaMemcpyHostToDevice, s));
+  if ((st = afd_ffn_forward(h, h->hin, T, h->hout, stream)) != AFD_OK) return st;
+  AFD_CUDA(h, cudaMemcpyAsync(out_host, h->hout, bytes, cudaMemcpyDeviceToHost, s));
+  AFD_CUDA(h, cudaStreamSynchronize(s));
+  return AFD_OK;
+}
+
+int afd_ffn_set_stage_events(afd_ffn_handle* h, void* const* events, int32_t n_events) {
+  if (!h || n_events < 0 || n_events > AFD_FFN_NUM_STAGES + 1) return AFD_ERR_INVALID_ARG;
+  if (n_events > 0 && !events) return AFD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i) h->events[i] = static_cast<cudaEvent_t>(events[i]);
+  h->n_events = n_events;
+  return AFD_OK;
+}
+
+int afd_ffn_get_error(afd_ffn_handle* h) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  AFD_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  int word = 0;
+  AFD_CUDA(h, cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  AFD_CUDA(h, cudaMemset(h->err, 0, sizeof(int)));
+  if (word & kErrTimeout) return AFD_ERR_DEVICE_TIMEOUT;
+  if (word) return AFD_ERR_DEVICE_FLAG;
+  return AFD_OK;
+}
+
+}  // extern "C"

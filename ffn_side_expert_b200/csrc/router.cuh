@@ -1,0 +1,141 @@
+// router.cuh -- router logits, top-k selection and gate weights.
+//
+// The FFN path is dominated by the routing computation and the exchange of hidden states
+// (vLLM AFD Plugin, Attention-FFN 解耦的原理); the router picks a few of the layer's many
+// experts per token (LLM 推理提速: Attention与FFN分离AFD方, 一个在啃带宽，一个在吃算力).
+// Reading taken: l = hidden . Wr^T (+ bias) in fp32, the k largest logits in descending
+// order (ties to the lower expert), w = softmax over the selected logits.
+//
+// router_logits_kernel: fp32 FMA GEMM, 64 tokens x 64 experts per CTA, 4x4 outputs per
+// thread, K tiles of 32 staged in shared memory, optionally split over K into partial sums
+// (deterministic: the top-k kernel adds the partials in split order).
+// router_topk_kernel: one warp per token; the logits of E <= 256 experts sit 8 per lane,
+// k rounds of warp arg-max reductions pick the experts, a warp sum normalises the weights.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace afd {
+
+constexpr int kRtTok = 64, kRtExp = 64, kRtK = 32;
+
+__global__ void __launch_bounds__(256)
+router_logits_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr,
+                     float* __restrict__ part, int T, int H, int E, int ktiles_per_split) {
+  __shared__ float xs[kRtK][kRtTok + 4];
+  __shared__ float ws[kRtK][kRtExp + 4];
+  const int t0 = blockIdx.y * kRtTok;
+  const int e0 = blockIdx.x * kRtExp;
+  const int kt0 = blockIdx.z * ktiles_per_split;
+  const int kt1 = min(H / kRtK, kt0 + ktiles_per_split);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int lr = threadIdx.x >> 2, lc = (threadIdx.x & 3) * 8;
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int kt = kt0; kt < kt1; ++kt) {
+    const int kb = kt * kRtK;
+    {  // 64 tokens x 32 hidden values, one 16-byte load per thread
+      const int t = t0 + lr;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t < T) v = *reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H + kb + lc);
+      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xs[lc + i][lr] = __bfloat162float(hv[i]);
+    }
+    {  // 64 experts x 32 hidden values of the fp32 router, two 16-byte loads per thread
+      const int e = e0 + lr;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+      if (e < E) {
+        const float4* p = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H + kb + lc);
+        a = p[0];
+        b = p[1];
+      }
+      ws[lc + 0][lr] = a.x; ws[lc + 1][lr] = a.y; ws[lc + 2][lr] = a.z; ws[lc + 3][lr] = a.w;
+      ws[lc + 4][lr] = b.x; ws[lc + 5][lr] = b.y; ws[lc + 6][lr] = b.z; ws[lc + 7][lr] = b.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kRtK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+    float* dst = part + (static_cast<size_t>(blockIdx.z) * T + t) * E;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) dst[e] = acc[i][j];
+    }
+  }
+}
+
+// One warp per token.  part: [nsplit][T][E] partial logits; bias: [E] or nullptr.
+__global__ void __launch_bounds__(256)
+router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __restrict__ bias,
+                   int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float v[8];
+  unsigned taken = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    float s = -INFINITY;
+    if (e < E) {
+      s = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) s += part[(static_cast<size_t>(sp) * T + t) * E + e];
+      if (bias) s += bias[e];
+    }
+    v[i] = s;
+  }
+  int my_e = -1;
+  float my_v = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // expert index grows with i: the first best is the lowest
+      const int e = lane + 32 * i;
+      if (e < E && !(taken >> i & 1u) && (v[i] > bv || (be == 0x7fffffff && v[i] == bv))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) { my_e = (be == 0x7fffffff) ? -1 : be; my_v = bv; }
+  }
+  const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+  const float z = (lane < k) ? expf(my_v - vmax) : 0.f;
+  const float sum = warp_sum(z);
+  if (lane < k) {
+    idx[static_cast<size_t>(t) * k + lane] = my_e;
+    w[static_cast<size_t>(t) * k + lane] = z / sum;
+  }
+}
+
+}  // namespace afd

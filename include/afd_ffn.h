@@ -1,0 +1,153 @@
+/*
+ * afd_ffn.h -- C ABI of libafd_ffn.so, the FFN-service MoE layer of Attention-FFN
+ * Disaggregation on one NVIDIA B200 (sm_100a).
+ *
+ * What the layer is.  In an A/F split the FFN service receives each layer's post-attention
+ * hidden states and returns the layer's FFN output (vLLM AFD Plugin page, section 系統架構,
+ * "2. FFN Service": a background loop receives activations, runs compute_ffn_output() and
+ * sends the result back).  For an MoE model that output is the routed expert layer: a router
+ * picks a few of many experts per token (LLM 推理提速: Attention与FFN分离AFD方, section 一个在
+ * 啃带宽，一个在吃算力), the hidden state is dispatched to them, each expert is a large matrix
+ * product, and the outputs are combined back per token (A/F 分离, sections 为什么要拆 and 机制).
+ *
+ * Readings where the pages are silent (the pages print no router or expert formula):
+ *   logits  l[t,e]  = sum_h hidden[t,h] * router_w[e,h] (+ router_bias[e])   fp32
+ *   idx[t,0..k-1]   = the k largest logits, descending, ties to the lower expert
+ *   w[t,j]          = softmax of the selected logits (= renormalised full softmax)
+ *   expert e        : y = (silu(x Wg_e^T) * (x Wu_e^T)) W2_e^T,  silu(z) = z / (1 + e^-z)
+ *   out[t]          = sum_j w[t,j] * y_{idx[t,j]}(x_t) + y_shared(x_t)      (shared: n_shared = 1)
+ * W8A8: each hidden row and each SwiGLU output row is quantised to e4m3 with one fp32 scale
+ * (row amax / 448, 1 for an all-zero row, round to nearest even, saturating) before the
+ * product that consumes it; weights arrive as e4m3 with one fp32 scale per output channel.
+ *
+ * Conventions for every entry point below.
+ *   - Return value: AFD_OK (0) or a negative AFD_ERR_* status; nothing is thrown.  Checks
+ *     that need no device run first and fail immediately (the FFN side fails fast when it is
+ *     driven wrongly: Separar Attention de FFN page, section "Ejecutarlo en una sola máquina").
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless stated otherwise.
+ *     Weight pointers are borrowed: they must stay valid and unchanged until destroy.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *     returns without a host synchronisation, except where stated.  The calling thread's
+ *     current device must be the device the handle was created on.
+ *   - One handle owns one device workspace sized for T_max tokens.  Calls on one handle must
+ *     not overlap in time (use one stream per handle, or synchronise between streams).
+ *   - Data the device finds invalid (an expert index outside [0,E), a position outside the
+ *     dispatched range) is skipped and recorded in the handle's device error word; read it
+ *     with afd_ffn_get_error.  No kernel traps.
+ *   - Layouts are row-major.  bf16 is IEEE bfloat16; e4m3 is the OCP "fn" variant.
+ */
+#ifndef AFD_FFN_H
+#define AFD_FFN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------- */
+#define AFD_OK                  0
+#define AFD_ERR_INVALID_ARG    (-1)  /* NULL / misaligned pointer, bad size or config field   */
+#define AFD_ERR_UNSUPPORTED    (-2)  /* config outside what the kernels implement             */
+#define AFD_ERR_T_TOO_LARGE    (-3)  /* T > T_max of the handle                               */
+#define AFD_ERR_CUDA           (-4)  /* a CUDA runtime/driver call failed: afd_ffn_last_cuda_error */
+#define AFD_ERR_DEVICE_FLAG    (-5)  /* afd_ffn_get_error: kernels skipped invalid data        */
+#define AFD_ERR_DEVICE_TIMEOUT (-6)  /* afd_ffn_get_error: a bounded on-device wait gave up    */
+#define AFD_ERR_NO_DEVICE      (-7)  /* no sm_100 device current                               */
+
+/* ---- configuration ---------------------------------------------------------------- */
+typedef enum { AFD_DT_BF16 = 0, AFD_DT_FP8_E4M3 = 1 } afd_dtype;
+
+typedef struct {
+    int32_t T_max;           /* largest micro-batch any call will pass, >= 1                  */
+    int32_t H;               /* hidden size, multiple of 256                                  */
+    int32_t E;               /* routed experts, 1..256                                        */
+    int32_t k;               /* experts per token, 1..min(E, 32)                              */
+    int32_t I;               /* expert intermediate size, multiple of 128                     */
+    int32_t n_shared;        /* shared experts: 0 or 1                                        */
+    int32_t weight_dtype;    /* afd_dtype: AFD_DT_BF16 or AFD_DT_FP8_E4M3                     */
+    int32_t act_dtype;       /* afd_dtype: must equal weight_dtype                            */
+    int32_t has_router_bias; /* 0 or 1                                                        */
+} afd_ffn_cfg;
+
+typedef struct {             /* all DEVICE pointers, 16-byte aligned, borrowed, never written */
+    const float *router_w;    /* [E][H] fp32                                                  */
+    const float *router_bias; /* [E] fp32, or NULL when has_router_bias == 0                  */
+    const void  *w13;         /* [E+n_shared][2I][H] bf16 or e4m3: rows 0..I-1 gate, I..2I-1 up;
+                                 the shared expert is index E                                  */
+    const void  *w2;          /* [E+n_shared][H][I] bf16 or e4m3 (down projection)            */
+    const float *w13_scale;   /* e4m3 only: [E+n_shared][2I] per-output-channel scales         */
+    const float *w2_scale;    /* e4m3 only: [E+n_shared][H]                                    */
+} afd_ffn_weights;
+
+typedef struct afd_ffn_handle afd_ffn_handle;
+
+/* Create a handle on the current device: validates cfg and weights (host-side checks come
+ * first and touch no device), allocates the workspace for T_max tokens and encodes the TMA
+ * descriptors of the weights.  *out receives the handle (NULL on failure).  Synchronous. */
+int afd_ffn_create(const afd_ffn_cfg *cfg, const afd_ffn_weights *weights, afd_ffn_handle **out);
+
+/* Free the workspace and the handle (after synchronising the device).  NULL is a no-op. */
+void afd_ffn_destroy(afd_ffn_handle *h);
+
+/* Router, top-k and gate weights.  hidden [T][H] bf16 -> topk_idx [T][k] int32 (descending
+ * logit order) and topk_w [T][k] fp32 (softmax over the selected logits).  0 <= T <= T_max. */
+int afd_ffn_route(afd_ffn_handle *h, const void *hidden, int32_t T,
+                  int32_t *topk_idx, float *topk_w, void *stream);
+
+/* Dispatch order and dispatched rows.  From topk_idx [T][k]:
+ *   counts [E]      rows per expert
+ *   offsets[E+1]    exclusive prefix sum of counts (offsets[E] = number of valid pairs)
+ *   pos    [T][k]   dispatched row of pair (t,j): expert-major, ascending t inside an expert;
+ *                   -1 for a pair whose expert is outside [0,E) (device error word set)
+ *   src    [T*k]    token of each dispatched row
+ * and fills the handle's internal dispatched-row buffer (hidden rows in pos order, then all
+ * T rows for the shared expert; e4m3 + per-row scale in W8A8) used by afd_ffn_expert_gemm. */
+int afd_ffn_permute(afd_ffn_handle *h, const void *hidden, const int32_t *topk_idx, int32_t T,
+                    int32_t *counts, int32_t *offsets, int32_t *pos, int32_t *src, void *stream);
+
+/* Expert FFNs on the rows dispatched by the last afd_ffn_permute of this handle, grouped by
+ * `offsets` [E+1] (device).  Writes the handle's internal output rows; when non-NULL also
+ * copies them out: Y [T*k][H] fp32 (row p = the output of dispatched row p, unweighted) and
+ * Ys [T][H] fp32 (shared expert; must be NULL when n_shared == 0). */
+int afd_ffn_expert_gemm(afd_ffn_handle *h, const int32_t *offsets, int32_t T,
+                        float *Y, float *Ys, void *stream);
+
+/* Weighted combine of the handle's internal expert outputs:
+ * out[t] = sum_j topk_w[t][j] * Y[pos[t][j]] + Ys[t], fp32 sum in j order, bf16 out [T][H]. */
+int afd_ffn_combine(afd_ffn_handle *h, const float *topk_w, const int32_t *pos, int32_t T,
+                    void *out, void *stream);
+
+/* The whole layer: hidden [T][H] bf16 -> out [T][H] bf16 (route, permute, expert GEMMs,
+ * combine).  No host synchronisation, no allocation: capturable in a CUDA graph. */
+int afd_ffn_forward(afd_ffn_handle *h, const void *hidden, int32_t T, void *out, void *stream);
+
+/* The whole layer on HOST buffers: copies hidden_host [T][H] bf16 to the device, runs
+ * afd_ffn_forward, copies the result to out_host [T][H] bf16, and synchronises `stream`
+ * before returning.  Pinned host memory gives the fastest copies. */
+int afd_ffn_forward_host(afd_ffn_handle *h, const void *hidden_host, int32_t T, void *out_host,
+                         void *stream);
+
+/* Optional stage timing: n_events cudaEvent_t handles (owned by the caller) that
+ * afd_ffn_forward records on its stream before each stage and after the last one.  Stages,
+ * in order: router logits, top-k, dispatch order, row gather, GEMM schedule, gate/up GEMM,
+ * activation quantisation (W8A8 only; empty otherwise), down GEMM, combine -- so
+ * AFD_FFN_NUM_STAGES + 1 events.  n_events = 0 (events NULL) turns it off. */
+#define AFD_FFN_NUM_STAGES 9
+int afd_ffn_set_stage_events(afd_ffn_handle *h, void *const *events, int32_t n_events);
+
+/* Synchronise the handle's last stream, return AFD_OK / AFD_ERR_DEVICE_FLAG /
+ * AFD_ERR_DEVICE_TIMEOUT from the device error word, and clear it. */
+int afd_ffn_get_error(afd_ffn_handle *h);
+
+/* The cudaError_t behind the last AFD_ERR_CUDA of this handle (0 if none; h may be NULL for
+ * errors of afd_ffn_create, which are kept per thread). */
+int afd_ffn_last_cuda_error(const afd_ffn_handle *h);
+
+/* Static description of a status code. */
+const char *afd_ffn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AFD_FFN_H */

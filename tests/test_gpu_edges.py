@@ -1,0 +1,154 @@
+"""Edge cases of the GPU path: empty and ragged micro-batches, T_max, T beyond T_max,
+invalid expert indices, degenerate routings (one expert, all experts, every token on the same
+experts), several N tiles of one expert, the shared expert and the W8A8 path at small sizes.
+Each case is compared with the fp64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import ffn_side_expert_b200 as afd
+import synth
+from layer_support import BF16_TOL, FP8_TOL, Layer, rel_max_err, to64
+from oracle import moe
+
+pytestmark = pytest.mark.gpu
+
+
+def _redraws(cfg, T=None):
+    """Margin redraws for an ad-hoc workload, found with the oracle."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden"))
+    from make_margin_redraws import find_redraws
+    return find_redraws(cfg, T=T)
+
+
+def _check_layer(L, T, tol=BF16_TOL):
+    out = L.forward(T)
+    torch.cuda.synchronize()
+    assert L.mod.get_error() == 0
+    ref = moe.forward(L.hidden[:T], L.Wr, L.bias, L.expert_fn, L.cfg.E, L.cfg.k, L.cfg.S, fp8=L.fp8)
+    idx, _ = L.route(T)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    err = rel_max_err(to64(out), ref["out"])
+    assert err <= tol, err
+    return out
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    L = Layer(synth.CONFIGS["tiny"])
+    yield L
+    L.close()
+
+
+def test_empty_batch_is_a_no_op(tiny):
+    out = torch.full((1, tiny.cfg.H), 3.0, dtype=torch.bfloat16, device="cuda")
+    assert afd.afd_ffn_forward(tiny.mod.h, tiny.h, 0, out) == afd.AFD_OK
+    torch.cuda.synchronize()
+    assert torch.all(out == 3.0)
+    assert tiny.mod.get_error() == 0
+
+
+@pytest.mark.parametrize("T", [1, 2, 37, 63, 64])
+def test_ragged_and_full_batches(tiny, T):
+    _check_layer(tiny, T)
+
+
+def test_T_beyond_T_max_fails_fast(tiny):
+    out = torch.empty((65, tiny.cfg.H), dtype=torch.bfloat16, device="cuda")
+    assert afd.afd_ffn_forward(tiny.mod.h, tiny.h, 65, out) == afd.AFD_ERR_T_TOO_LARGE
+    assert afd.afd_ffn_forward(tiny.mod.h, tiny.h, -1, out) == afd.AFD_ERR_INVALID_ARG
+
+
+def test_invalid_expert_indices_are_skipped_and_flagged(tiny):
+    _, ridx, _ = tiny.oracle_routing()
+    bad = ridx.copy()
+    bad[3, 1] = tiny.cfg.E          # out of range
+    bad[10, 0] = -5
+    counts, offsets, pos, src = tiny.permute(torch.from_numpy(bad).cuda())
+    torch.cuda.synchronize()
+    assert tiny.mod.get_error() == afd.AFD_ERR_DEVICE_FLAG
+    assert tiny.mod.get_error() == afd.AFD_OK               # cleared by the read
+    rc, ro, rp, rs = moe.permute(bad, tiny.cfg.E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(pos.cpu().numpy(), rp)
+    assert np.array_equal(src.cpu().numpy()[:len(rs)], rs)
+
+
+def test_combine_flags_positions_out_of_range(tiny):
+    idx, w = tiny.route()
+    counts, offsets, pos, src = tiny.permute(idx)
+    tiny.expert_gemm(offsets, idx.shape[0])
+    pos2 = pos.clone()
+    pos2[0, 0] = 10 ** 6
+    tiny.combine(w, pos2, idx.shape[0])
+    torch.cuda.synchronize()
+    assert tiny.mod.get_error() == afd.AFD_ERR_DEVICE_FLAG
+
+
+def test_every_token_on_the_same_experts():
+    # a large bias on experts 2 and 5 sends every token there: two groups of T rows, the
+    # other experts empty
+    cfg = synth.MoEConfig("skewed", T=64, H=256, E=8, k=2, I=512, seed=21)
+    bias = np.zeros(cfg.E, dtype=np.float32)
+    bias[2], bias[5] = 60.0, 40.0
+    L = Layer(cfg, bias=torch.from_numpy(bias), redraws={})
+    try:
+        out = _check_layer(L, cfg.T)
+        idx, _ = L.route()
+        assert set(np.unique(idx.cpu().numpy())) == {2, 5}
+    finally:
+        L.close()
+
+
+def test_single_expert_top1_is_dense_ffn():
+    cfg = synth.MoEConfig("e1k1", T=40, H=256, E=1, k=1, I=256, seed=22)
+    L = Layer(cfg, redraws={})
+    try:
+        out = L.forward()
+        w13, w2 = moe.expert_weights_f64(L.expert_fn(0))
+        dense, _ = moe.swiglu_ffn(moe._f64(L.hidden), w13, w2)
+        assert rel_max_err(to64(out), dense) <= BF16_TOL
+    finally:
+        L.close()
+
+
+def test_all_experts_selected_with_shared_expert():
+    cfg = synth.MoEConfig("kE", T=48, H=256, E=4, k=4, I=128, S=1, seed=23)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, cfg.T)
+    finally:
+        L.close()
+
+
+def test_wide_tiles_with_several_n_tiles_per_expert():
+    # T*k > 32 E selects the wide tiles (N up to 256); 600 tokens over 2 experts gives each
+    # expert ~300 rows: two N tiles, the second ragged
+    cfg = synth.MoEConfig("wide", T=600, H=256, E=2, k=1, I=256, S=1, seed=24)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, cfg.T)
+    finally:
+        L.close()
+
+
+@pytest.mark.parametrize("T", [64, 23])
+def test_w8a8_small(T):
+    cfg = synth.MoEConfig("fp8s", T=64, H=512, E=8, k=2, I=256, S=1, dtype="fp8", seed=25)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, T, tol=FP8_TOL)
+    finally:
+        L.close()
+
+
+def test_w8a8_wide_tiles():
+    cfg = synth.MoEConfig("fp8w", T=512, H=256, E=4, k=2, I=256, S=1, dtype="fp8", seed=26)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, cfg.T, tol=FP8_TOL)
+    finally:
+        L.close()
