@@ -162,9 +162,20 @@ def cpu_baseline(cfg, hidden, Wr, bias, ex, budget_s=15.0) -> dict:
                       f"(routing, {cfg.k} experts + {cfg.S} shared per token), {spent:.1f} s"}
 
 
+def workload(args):
+    cfg = synth.CONFIGS[args.config]
+    over = {k: v for k, v in (("T", args.T), ("E", args.E)) if v is not None}
+    return cfg.with_(**over) if over else cfg
+
+
+def workload_label(args) -> str:
+    over = [f"{k}={v}" for k, v in (("T", args.T), ("E", args.E)) if v is not None]
+    return args.config + (f"[{','.join(over)}]" if over else "")
+
+
 def run_ours(args, rank, world, local_rank):
     import ffn_side_expert_b200 as afd
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     hidden, Wr, bias, ex, dev = build_inputs(cfg, device)
@@ -265,8 +276,8 @@ def report_ours(args, world, r) -> dict:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3" if cfg.dtype == "fp8" else "bf16", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
-                   "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed,
+        "config": {"workload": workload_label(args), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
+                   "I": cfg.I, "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (expert weights 22.6 GB >> 126 MB)"},
         "roofline": {"bound": "hbm", "kernel": "grouped_gemm gate/up + SwiGLU",
@@ -296,7 +307,7 @@ def run_reference(args, rank, world):
     from oracle import moe
     if rank != 0:
         return None
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     hidden = synth.gen_hidden(cfg)
     Wr, bias = synth.gen_router(cfg)
     n = max(1, int(args.ref_tokens))
@@ -322,8 +333,8 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * per_tok * cfg.T, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
-                   "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed},
+        "config": {"workload": workload_label(args), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
+                   "I": cfg.I, "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n} token(s) of the {cfg.name} micro-batch per step, full fp64 layer "
                                    f"(expert weights drawn before timing); ms_per_step scaled to T={cfg.T}"},
@@ -341,6 +352,10 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=1, help="reference arm: tokens per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None,
+                    help="profiling only: override the micro-batch size (a smaller case of the same kernels)")
+    ap.add_argument("--E", type=int, default=None,
+                    help="profiling only: override the number of routed experts")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

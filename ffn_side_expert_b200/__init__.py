@@ -156,9 +156,16 @@ def afd_ffn_forward_host(h, hidden_host, T, out_host, stream=None) -> int:
 
 
 def afd_ffn_set_stage_events(h, events) -> int:
-    """events: sequence of torch.cuda.Event (AFD_FFN_NUM_STAGES + 1 of them) or None."""
+    """events: sequence of torch.cuda.Event (AFD_FFN_NUM_STAGES + 1 of them) or None.
+
+    torch creates an event's CUDA handle at its first record; events not yet created are
+    recorded once on the current stream here so that the library receives real handles.
+    """
     if not events:
         return _lib.afd_ffn_set_stage_events(h, None, 0)
+    for e in events:
+        if not e.cuda_event:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     return _lib.afd_ffn_set_stage_events(h, arr, len(events))
 

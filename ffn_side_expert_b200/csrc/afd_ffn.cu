@@ -25,11 +25,15 @@ using namespace afd;
 
 namespace {
 
-// Two tile shapes of the grouped GEMM: "narrow" for decode micro-batches (a few rows per
+// Two tile shapes of the grouped GEMMs: "narrow" for decode micro-batches (a few rows per
 // expert: N <= 32, a deep ring of small stages, double-buffered TMEM) and "wide" for large
-// micro-batches (N <= 256, the widest MMA; three 64 KB stages).
-constexpr int kNarrowBN = 32, kNarrowStages = 6;
-constexpr int kWideBN = 256, kWideStages = 3;
+// micro-batches (N <= 256, the widest MMA, three 64 KB stages).  The bf16 down GEMM reads two
+// activation planes (hi, lo) per stage, so its wide shape is N <= 128 (still three stages).
+struct Shape {
+  int bn1, bn2;  // N tile of the gate/up and of the down GEMM
+};
+constexpr int kNarrowBN = 32, kNarrowStages = 6, kNarrowSplitStages = 5;
+constexpr int kWideBN = 256, kWideStages = 3, kWideSplitBN = 128;
 
 thread_local int g_create_cuda_error = 0;
 
@@ -59,7 +63,7 @@ struct afd_ffn_handle {
   int32_t* ub2 = nullptr;
   uint8_t* xp = nullptr;     // dispatched rows [R_max][H] bf16 / e4m3
   float* xscale = nullptr;   // [R_max]
-  void* act = nullptr;       // [R_max][I] bf16 (or fp32 in W8A8)
+  void* act = nullptr;       // [2][R_max][I] bf16 hi/lo planes (or [R_max][I] fp32 in W8A8)
   uint8_t* actq = nullptr;   // W8A8: [R_max][I] e4m3
   float* ascale = nullptr;   // W8A8: [R_max]
   float* Y = nullptr;        // [R_max][H] fp32
@@ -145,29 +149,60 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool FP8, int MODE>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8, MODE>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, STAGES>());
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8, MODE, SPLIT>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, STAGES, SPLIT>());
+}
+
+// (gate/up, down) kernel pairs of each path and tile shape
+template <bool FP8, bool NARROW>
+struct GemmPair;
+template <>
+struct GemmPair<false, true> {  // bf16 decode
+  static constexpr int bn1 = kNarrowBN, st1 = kNarrowStages, bn2 = kNarrowBN, st2 = kNarrowSplitStages;
+  static constexpr bool split = true;
+};
+template <>
+struct GemmPair<false, false> {  // bf16 large micro-batch
+  static constexpr int bn1 = kWideBN, st1 = kWideStages, bn2 = kWideSplitBN, st2 = kWideStages;
+  static constexpr bool split = true;
+};
+template <>
+struct GemmPair<true, true> {  // W8A8 decode
+  static constexpr int bn1 = kNarrowBN, st1 = kNarrowStages, bn2 = kNarrowBN, st2 = kNarrowStages;
+  static constexpr bool split = false;
+};
+template <>
+struct GemmPair<true, false> {  // W8A8 large micro-batch
+  static constexpr int bn1 = kWideBN, st1 = kWideStages, bn2 = kWideBN, st2 = kWideStages;
+  static constexpr bool split = false;
+};
+
+template <bool FP8, bool NARROW>
+cudaError_t set_pair_attrs() {
+  using P = GemmPair<FP8, NARROW>;
+  cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false>();
+  if (e != cudaSuccess) return e;
+  return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split>();
 }
 
 template <bool FP8>
 cudaError_t set_all_gemm_attrs() {
-  cudaError_t e;
-  if ((e = set_gemm_attr<kNarrowBN, kNarrowStages, FP8, 0>()) != cudaSuccess) return e;
-  if ((e = set_gemm_attr<kNarrowBN, kNarrowStages, FP8, 1>()) != cudaSuccess) return e;
-  if ((e = set_gemm_attr<kWideBN, kWideStages, FP8, 0>()) != cudaSuccess) return e;
-  return set_gemm_attr<kWideBN, kWideStages, FP8, 1>();
+  cudaError_t e = set_pair_attrs<FP8, true>();
+  if (e != cudaSuccess) return e;
+  return set_pair_attrs<FP8, false>();
 }
 
-template <int BN, int STAGES, bool FP8, int MODE>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT>
 void launch_gemm(const afd_ffn_handle* h, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args,
                  cudaStream_t s) {
-  grouped_gemm_kernel<BN, STAGES, FP8, MODE>
-      <<<h->num_sms, 192, gemm_smem_bytes<BN, STAGES>(), s>>>(a, b, args);
+  grouped_gemm_kernel<BN, STAGES, FP8, MODE, SPLIT>
+      <<<h->num_sms, 192, gemm_smem_bytes<BN, STAGES, SPLIT>(), s>>>(a, b, args);
 }
 
 void record(afd_ffn_handle* h, int stage, cudaStream_t s) {
+  // a failure here surfaces through the cudaGetLastError check that ends each stage
   if (h->n_events > stage) cudaEventRecord(h->events[stage], s);
 }
 
@@ -203,8 +238,9 @@ int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T
   return AFD_OK;
 }
 
-template <int BN, int STAGES, bool FP8>
+template <bool FP8, bool NARROW>
 void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
+  using P = GemmPair<FP8, NARROW>;
   const afd_ffn_cfg& c = h->cfg;
   const int R = T * c.k + T;
   GemmArgs g1{};
@@ -218,11 +254,12 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g1.second_off = c.I;
   g1.out = h->act;
   g1.out_ld = c.I;
+  g1.lo_rows = h->R_max;
   g1.a_scale = h->w.w13_scale;
   g1.b_scale = h->xscale;
   g1.err = h->err;
   record(h, 5, s);
-  launch_gemm<BN, STAGES, FP8, 0>(h, h->tm_w13, h->tm_xp, g1, s);
+  launch_gemm<P::bn1, P::st1, FP8, 0, false>(h, h->tm_w13, h->tm_xp, g1, s);
   record(h, 6, s);
   if (FP8) quantize_act_kernel<<<R, 256, 0, s>>>(static_cast<const float*>(h->act), c.I, h->actq, h->ascale);
   GemmArgs g2 = g1;
@@ -236,22 +273,29 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g2.a_scale = h->w.w2_scale;
   g2.b_scale = h->ascale;
   record(h, 7, s);
-  launch_gemm<BN, STAGES, FP8, 1>(h, h->tm_w2, h->tm_act, g2, s);
+  launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(h, h->tm_w2, h->tm_act, g2, s);
 }
 
 int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   const bool narrow = use_narrow(h, T);
-  const int bn = narrow ? kNarrowBN : kWideBN;
-  record(h, 4, s);
-  build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn, c.I / 128, c.H / 256, h->grp_rows,
-                                          h->grp_base, h->ub1, h->ub2, h->err);
+  int bn1, bn2;
   if (h->fp8) {
-    if (narrow) run_gemms<kNarrowBN, kNarrowStages, true>(h, T, s);
-    else run_gemms<kWideBN, kWideStages, true>(h, T, s);
+    bn1 = narrow ? GemmPair<true, true>::bn1 : GemmPair<true, false>::bn1;
+    bn2 = narrow ? GemmPair<true, true>::bn2 : GemmPair<true, false>::bn2;
   } else {
-    if (narrow) run_gemms<kNarrowBN, kNarrowStages, false>(h, T, s);
-    else run_gemms<kWideBN, kWideStages, false>(h, T, s);
+    bn1 = narrow ? GemmPair<false, true>::bn1 : GemmPair<false, false>::bn1;
+    bn2 = narrow ? GemmPair<false, true>::bn2 : GemmPair<false, false>::bn2;
+  }
+  record(h, 4, s);
+  build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn1, bn2, c.I / 128, c.H / 256,
+                                          h->grp_rows, h->grp_base, h->ub1, h->ub2, h->err);
+  if (h->fp8) {
+    if (narrow) run_gemms<true, true>(h, T, s);
+    else run_gemms<true, false>(h, T, s);
+  } else {
+    if (narrow) run_gemms<false, true>(h, T, s);
+    else run_gemms<false, false>(h, T, s);
   }
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
@@ -372,7 +416,7 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
       {reinterpret_cast<void**>(&h->ub2), static_cast<size_t>(h->G + 1) * 4},
       {reinterpret_cast<void**>(&h->xp), R * c.H * wb},
       {reinterpret_cast<void**>(&h->xscale), R * 4},
-      {&act_p, R * c.I * (h->fp8 ? 4 : 2)},
+      {&act_p, R * c.I * 4},  // fp32 (W8A8) or two bf16 planes (hi, lo)
       {reinterpret_cast<void**>(&h->actq), h->fp8 ? R * c.I : 0},
       {reinterpret_cast<void**>(&h->ascale), R * 4},
       {reinterpret_cast<void**>(&h->Y), R * c.H * 4},
@@ -397,7 +441,8 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   bool ok = encode_2d(&h->tm_w13, weights->w13, h->fp8, c.H, G * 2 * c.I, 128) &&
             encode_2d(&h->tm_w2, weights->w2, h->fp8, c.I, G * c.H, 128) &&
             encode_2d(&h->tm_xp, h->xp, h->fp8, c.H, R, 16) &&
-            encode_2d(&h->tm_act, h->fp8 ? static_cast<const void*>(h->actq) : h->act, h->fp8, c.I, R, 16);
+            encode_2d(&h->tm_act, h->fp8 ? static_cast<const void*>(h->actq) : h->act, h->fp8, c.I,
+                      h->fp8 ? R : 2 * R, 16);
   if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
   if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
@@ -504,6 +549,8 @@ int afd_ffn_forward_host(afd_ffn_handle* h, const void* hidden_host, int32_t T, 
 int afd_ffn_set_stage_events(afd_ffn_handle* h, void* const* events, int32_t n_events) {
   if (!h || n_events < 0 || n_events > AFD_FFN_NUM_STAGES + 1) return AFD_ERR_INVALID_ARG;
   if (n_events > 0 && !events) return AFD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return AFD_ERR_INVALID_ARG;
   for (int i = 0; i < n_events; ++i) h->events[i] = static_cast<cudaEvent_t>(events[i]);
   h->n_events = n_events;
   return AFD_OK;

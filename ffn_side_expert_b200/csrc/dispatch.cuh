@@ -195,11 +195,11 @@ quantize_act_kernel(const float* __restrict__ act32, int I, uint8_t* __restrict_
 }
 
 // GEMM schedule from the group offsets: group g < E is expert g (rows offsets[g]..offsets[g+1]),
-// group E is the shared expert (rows shared_base .. shared_base + T).  Each group contributes
-// ceil(rows / bn) * mt tile units to each GEMM; unit bases are exclusive prefix sums.
-// One CTA of 512 threads (G <= 257).
+// group E is the shared expert (rows T*k .. T*k + T).  Each group contributes
+// ceil(rows / bn1) * mt1 tile units to the gate/up GEMM and ceil(rows / bn2) * mt2 to the
+// down GEMM; unit bases are exclusive prefix sums.  One CTA of 512 threads (G <= 257).
 __global__ void __launch_bounds__(512)
-build_schedule_kernel(const int32_t* __restrict__ offsets, int E, int n_shared, int T, int k, int bn,
+build_schedule_kernel(const int32_t* __restrict__ offsets, int E, int n_shared, int T, int k, int bn1, int bn2,
                       int mt1, int mt2, int32_t* __restrict__ grp_rows, int32_t* __restrict__ grp_base,
                       int32_t* __restrict__ ub1, int32_t* __restrict__ ub2, int* err) {
   __shared__ int wsum1[16], wsum2[16];
@@ -218,8 +218,7 @@ build_schedule_kernel(const int32_t* __restrict__ offsets, int E, int n_shared, 
     rows = T;
     rbase = T * k;  // shared-expert rows follow the routed rows
   }
-  const int nt = (rows + bn - 1) / bn;
-  const int u1 = nt * mt1, u2 = nt * mt2;
+  const int u1 = (rows + bn1 - 1) / bn1 * mt1, u2 = (rows + bn2 - 1) / bn2 * mt2;
   const int i1 = warp_incl_scan(u1, lane), i2 = warp_incl_scan(u2, lane);
   if (lane == 31) { wsum1[warp] = i1; wsum2[warp] = i2; }
   __syncthreads();

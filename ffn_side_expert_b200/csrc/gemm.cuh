@@ -12,6 +12,13 @@
 // into two fp32 TMEM accumulators; the SwiGLU (MODE 0) and the scales of the W8A8 path are
 // applied in the epilogue straight from TMEM.
 //
+// bf16 path, two-term activations: the gate/up epilogue stores the fp32 SwiGLU output as
+// hi = bf16(act) and lo = bf16(act - hi) in two planes, and the down GEMM (SPLIT_B) multiplies
+// each weight tile by both and accumulates into one TMEM accumulator, so the activation enters
+// the down projection with ~2^-17 relative error instead of bf16's 2^-9 (the two-term bfloat16
+// split of Henry, Tang and Heinecke, "Leveraging the bfloat16 AI datatype for higher-precision
+// computations", 2019).  The only bf16 rounding left on the output path is the layer output.
+//
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep shared-memory
 // ring; warp 1 owns the TMEM allocation and its lane 0 issues tcgen05.mma; warps 2..5 are
 // the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).  Units are assigned round-robin over
@@ -40,15 +47,17 @@ struct GemmArgs {
   int second_off;            // row offset of a pair's second tile (I / 128)
   void* out;                 // MODE 0: act (bf16, or fp32 for W8A8) [R][I]; MODE 1: Y fp32 [R][H]
   int out_ld;                // elements per output row
+  int lo_rows;               // bf16 two-term activations: row offset of the lo plane (R_max)
   const float* a_scale;      // W8A8: per weight row [G * a_rows]
   const float* b_scale;      // W8A8: per token row [R]
   int* err;                  // device error word
 };
 
-template <int BN>
+template <int BN, bool SPLIT_B = false>
 struct GemmShape {
   static constexpr int kATile = 128 * 128;              // one 128-row x 128-byte weight tile
-  static constexpr int kStageBytes = 2 * kATile + BN * 128;
+  static constexpr int kBTile = BN * 128;               // up to BN token rows x 128 bytes
+  static constexpr int kStageBytes = 2 * kATile + (SPLIT_B ? 2 : 1) * kBTile;
   static constexpr int kNacc = (4 * BN <= 512) ? 2 : 1;  // accumulator sets in TMEM
   static constexpr int kColsUsed = kNacc * 2 * BN;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
@@ -57,9 +66,9 @@ struct GemmShape {
   static_assert(BN % 16 == 0 && BN <= 256, "N tile");
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SPLIT_B>
 constexpr int gemm_smem_bytes() {
-  return STAGES * GemmShape<BN>::kStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
+  return STAGES * GemmShape<BN, SPLIT_B>::kStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
 }
 
 __device__ __forceinline__ int find_group(const int32_t* __restrict__ unit_base, int G, int u) {
@@ -92,11 +101,12 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-template <int BN, int STAGES, bool FP8, int MODE>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B>
 __global__ void __launch_bounds__(192, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmArgs args) {
-  using S = GemmShape<BN>;
+  static_assert(!(SPLIT_B && (FP8 || MODE != 1)), "two-term B only for the bf16 down GEMM");
+  using S = GemmShape<BN, SPLIT_B>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
 
@@ -153,7 +163,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       const Unit w = decode_unit<BN>(args, u);
       const int ya = w.g * args.a_rows + w.mt * args.mt_stride;
-      const uint32_t tx = 2u * S::kATile + static_cast<uint32_t>(w.n16) * 128u;
+      const uint32_t tx = 2u * S::kATile + (SPLIT_B ? 2u : 1u) * static_cast<uint32_t>(w.n16) * 128u;
       for (int kc = 0; kc < kchunks; ++kc) {
         if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t st = base + s * S::kStageBytes;
@@ -163,6 +173,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tma_load_2d(st + S::kATile, &tmA, full_bar(s), x, ya + args.second_off, kEvictFirst);
         for (int r = 0; r < w.n16; r += 16)
           tma_load_2d(st + 2 * S::kATile + r * 128, &tmB, full_bar(s), x, w.row0 + r, kEvictLast);
+        if constexpr (SPLIT_B) {
+          for (int r = 0; r < w.n16; r += 16)
+            tma_load_2d(st + 2 * S::kATile + S::kBTile + r * 128, &tmB, full_bar(s), x,
+                        args.lo_rows + w.row0 + r, kEvictLast);
+        }
         ++issued;
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
@@ -200,6 +215,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           const uint32_t accum = (kc > 0 || kk > 0) ? 1u : 0u;
           tc_mma<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
           tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+          if constexpr (SPLIT_B) {  // the lo plane of the activations, same accumulators
+            const uint64_t dl = sw128_desc(st + 2 * S::kATile + S::kBTile);
+            tc_mma<FP8>(d0, da0 + 2 * kk, dl + 2 * kk, idesc, 1u);
+            tc_mma<FP8>(d1, da1 + 2 * kk, dl + 2 * kk, idesc, 1u);
+          }
         }
         tc_commit(empty_bar(s));  // frees the stage once these MMAs have read it
         if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -256,10 +276,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
             if constexpr (MODE == 0) {
               const float act = silu_f(v0) * v1;  // gate tile first, up tile second
-              if constexpr (FP8)
+              if constexpr (FP8) {
                 static_cast<float*>(args.out)[row * args.out_ld + wrow0] = act;
-              else
-                static_cast<__nv_bfloat16*>(args.out)[row * args.out_ld + wrow0] = __float2bfloat16_rn(act);
+              } else {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(act);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(act - __bfloat162float(hi));
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(args.out);
+                o[row * args.out_ld + wrow0] = hi;
+                o[(static_cast<size_t>(args.lo_rows) + row) * args.out_ld + wrow0] = lo;
+              }
             } else {
               float* y = static_cast<float*>(args.out) + row * args.out_ld;
               y[wrow0] = v0;

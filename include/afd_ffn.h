@@ -132,7 +132,8 @@ int afd_ffn_forward_host(afd_ffn_handle *h, const void *hidden_host, int32_t T, 
  * afd_ffn_forward records on its stream before each stage and after the last one.  Stages,
  * in order: router logits, top-k, dispatch order, row gather, GEMM schedule, gate/up GEMM,
  * activation quantisation (W8A8 only; empty otherwise), down GEMM, combine -- so
- * AFD_FFN_NUM_STAGES + 1 events.  n_events = 0 (events NULL) turns it off. */
+ * AFD_FFN_NUM_STAGES + 1 events, each already created (non-NULL; AFD_ERR_INVALID_ARG otherwise).
+ * n_events = 0 (events NULL) turns it off. */
 #define AFD_FFN_NUM_STAGES 9
 int afd_ffn_set_stage_events(afd_ffn_handle *h, void *const *events, int32_t n_events);
 
