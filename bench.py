@@ -33,6 +33,16 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up GEMM with the
+# decode tile shape, from the ncu capture in profiles/grouped_gemm_decode_T16_E16.md
+# (1 003 994 112 B for 272 weight-tile pairs: 17 expert groups x 16).  Traffic grows with the
+# distinct weight tiles streamed (the N tiles of one weight tile share it through L2), and it is
+# reported only while gemm.cuh is the source that was captured.
+MEASURED_TRAFFIC = {
+    "gemm_cuh_sha256": "6c6cb4e38901f8072a1cf0c878daf423345437ea7548b923ab12f5b5630f4a24",
+    "bytes_per_unit": 1003994112 / 272,
+}
 METRIC = "MoE-FFN tokens/s/layer"
 
 
@@ -58,8 +68,23 @@ def algorithmic(cfg, counts) -> dict:
     rows = T * k + S * T
     gemm13 = w13 + rows * H * b + rows * I * (4 if b == 1 else 2)
     flops = 6 * H * I * (T * k + S * T) + 2 * T * H * E
+    units = n * (I // 128)   # distinct gate/up weight-tile pairs streamed
     return {"weight_bytes": w13 + w2, "act_bytes": act, "flops": flops, "gemm13_bytes": gemm13,
-            "gemm13_flops": 4 * H * I * rows, "touched_experts": n}
+            "gemm13_flops": 4 * H * I * rows, "touched_experts": n, "gemm13_units_narrow": units}
+
+
+def gate_up_traffic(cfg, acct):
+    """Measured DRAM bytes per gate/up launch scaled to this workload, or None when the kernel
+    source changed since the capture or the launch uses another tile shape or dtype."""
+    import hashlib
+    path = os.path.join(ROOT, "ffn_side_expert_b200", "csrc", "gemm.cuh")
+    with open(path, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    narrow = cfg.T * cfg.k <= 32 * cfg.E
+    if sha != MEASURED_TRAFFIC["gemm_cuh_sha256"] or cfg.dtype != "bf16" or not narrow:
+        return None
+    units = acct["gemm13_units_narrow"]
+    return int(round(MEASURED_TRAFFIC["bytes_per_unit"] * units))
 
 
 def load_peaks():
@@ -282,7 +307,7 @@ def report_ours(args, world, r) -> dict:
                    "l2": "inputs larger than L2 (expert weights 22.6 GB >> 126 MB)"},
         "roofline": {"bound": "hbm", "kernel": "grouped_gemm gate/up + SwiGLU",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "frac": round(achieved / hbm, 4), "traffic": gate_up_traffic(cfg, acct),
                      "peak_source": f"{kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": acct["gemm13_bytes"],
                      "avg_launch_ms": round(g13_ms, 4)},
