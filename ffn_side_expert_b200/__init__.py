@@ -63,6 +63,7 @@ _SIGNATURES = {
     "afd_ffn_get_error": (ctypes.c_int, [_P]),
     "afd_ffn_last_cuda_error": (ctypes.c_int, [_P]),
     "afd_ffn_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "afd_ffn_route_static": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
 }
 
 
@@ -176,6 +177,16 @@ def afd_ffn_get_error(h) -> int:
 
 def afd_ffn_last_cuda_error(h) -> int:
     return _lib.afd_ffn_last_cuda_error(h)
+
+
+def afd_ffn_route_static(hidden, router_w, router_bias, T, H, E, k, topk_idx, topk_w, stream=None) -> int:
+    """Router without a handle or any allocation (scratch in a static device array); see the
+    declaration in include/afd_ffn.h for the size limit and the first-call set-up."""
+    return _lib.afd_ffn_route_static(_ptr(hidden), _ptr(router_w), _ptr(router_bias), T, H, E, k,
+                                     _ptr(topk_idx), _ptr(topk_w), _stream(stream))
+
+
+AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS = 1 << 20
 
 
 # ------------------------------------------------------------------ convenience wrapper

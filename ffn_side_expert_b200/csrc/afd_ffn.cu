@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "afd_ffn.h"
@@ -568,3 +569,65 @@ int afd_ffn_get_error(afd_ffn_handle* h) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------- allocation-free router
+// Scratch of afd_ffn_route_static: partial router logits.  File-scope device array; host code
+// only ever sees its host-side shadow, so the device address is looked up once per device.
+static __device__ __align__(256) float g_route_scratch[AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_route_scratch_mu;
+float* g_route_scratch_dev[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device (set-up on the first call).
+int route_scratch(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  if (dev < 0 || dev >= kMaxDevices) return AFD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+  if (!g_route_scratch_dev[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return cuda_fail(nullptr, e);
+    g_route_scratch_dev[dev] = static_cast<float*>(p);
+  }
+  *out = g_route_scratch_dev[dev];
+  return AFD_OK;
+}
+}  // namespace
+
+extern "C" int afd_ffn_route_static(const void* hidden, const float* router_w, const float* router_bias,
+                                    int32_t T, int32_t H, int32_t E, int32_t k, int32_t* topk_idx,
+                                    float* topk_w, void* stream) {
+  if (T < 0 || H < kRtK || H % kRtK != 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > 32)
+    return AFD_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * E > AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS) return AFD_ERR_UNSUPPORTED;
+  if (T == 0) return AFD_OK;
+  if (!hidden || !router_w || !topk_idx || !topk_w || !aligned16(hidden) || !aligned16(router_w))
+    return AFD_ERR_INVALID_ARG;
+  float* part = nullptr;
+  int st = route_scratch(&part);
+  if (st != AFD_OK) return st;
+  int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  int nsplit = 1, per = 1;
+  router_split(T, H, E, sms, &nsplit, &per);
+  const long long cap = AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS / (static_cast<long long>(T) * E);
+  if (nsplit > cap) {  // narrow the split of H until the partials fit the scratch
+    const int kt = H / kRtK;
+    per = (kt + static_cast<int>(cap) - 1) / static_cast<int>(cap);
+    nsplit = (kt + per - 1) / per;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid((E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
+  router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), router_w, part, T, H, E, per);
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}

@@ -148,6 +148,35 @@ int afd_ffn_last_cuda_error(const afd_ffn_handle *h);
 /* Static description of a status code. */
 const char *afd_ffn_strerror(int status);
 
+/* Router, top-k and gate weights with no handle and no allocation of any kind.
+ *
+ * This entry point has no counterpart on the pages; it exists for callers that cannot
+ * allocate device memory: a serving engine that owns every device byte through its own pool
+ * and caps it (a stray cudaMalloc there fails or breaks the engine's accounting), and the
+ * per-layer loop of an FFN service, where an allocation can synchronise the device in the
+ * middle of a pipelined micro-batch.  afd_ffn_create allocates a workspace, so such callers
+ * cannot use afd_ffn_route; this call computes the same thing (same kernels, same results
+ * within the router's fp32 rounding; identical when T*E*splits fits, see below).
+ *
+ * Inputs (device, caller-owned, 16-byte aligned): hidden [T][H] bf16, router_w [E][H] fp32,
+ * router_bias [E] fp32 or NULL.  Outputs: topk_idx [T][k] int32, topk_w [T][k] fp32.
+ * Sizes: 0 <= T, H a multiple of 32, 1 <= E <= 256, 1 <= k <= min(E, 32).
+ * Scratch: the partial router logits live in one static device array of
+ * AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS floats (4 MiB) that every GPU loading the library holds
+ * until the process exits.  T*E must not exceed it; larger problems return
+ * AFD_ERR_UNSUPPORTED before any device work (the split of the reduction over H is narrowed
+ * to fit, so results can differ from afd_ffn_route in the last fp32 bits when it is).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture on the device.
+ * Every call on a device shares the one array: calls that can overlap on the GPU (different
+ * streams without ordering between them) race on it and must be serialised by the caller.
+ * Nothing in the array needs clearing: each call overwrites every element it reads.
+ * CUDA failures return AFD_ERR_CUDA; the cudaError_t is afd_ffn_last_cuda_error(NULL). */
+#define AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS (1 << 20)
+int afd_ffn_route_static(const void *hidden, const float *router_w, const float *router_bias,
+                         int32_t T, int32_t H, int32_t E, int32_t k,
+                         int32_t *topk_idx, float *topk_w, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
