@@ -26,15 +26,12 @@ using namespace afd;
 
 namespace {
 
-// Two tile shapes of the grouped GEMMs: "narrow" for decode micro-batches (a few rows per
-// expert: N <= 32, a deep ring of small stages, double-buffered TMEM) and "wide" for large
-// micro-batches (N <= 256, the widest MMA, three 64 KB stages).  The bf16 down GEMM reads two
-// activation planes (hi, lo) per stage, so its wide shape is N <= 128 (still three stages).
-struct Shape {
-  int bn1, bn2;  // N tile of the gate/up and of the down GEMM
-};
-constexpr int kNarrowBN = 32, kNarrowStages = 6, kNarrowSplitStages = 5;
-constexpr int kWideBN = 256, kWideStages = 3, kWideSplitBN = 128;
+// Tile shapes of the grouped GEMMs (N tile and ring stages; GemmPair below): "narrow" for decode micro-batches (a few rows per expert, N <= 32) and "wide" for
+// large micro-batches (N <= 128).  The bf16 down GEMM reads two activation planes (hi, lo) per
+// token stage.  Both keep two accumulator sets in TMEM so the epilogue of one unit overlaps the
+// next unit's MMAs.
+// tensor-core router: N tile of 64 tokens, three weight planes per stage
+constexpr int kRouterBN = 64, kRouterStages = 3;
 
 thread_local int g_create_cuda_error = 0;
 
@@ -54,10 +51,13 @@ struct afd_ffn_handle {
   float* part = nullptr;
   int32_t* idx = nullptr;
   float* wts = nullptr;
+  void* wr_planes = nullptr; // [3][E][H] bf16: router weights hi, mid, lo
   int32_t* counts = nullptr;
   int32_t* offsets = nullptr;
   int32_t* pos = nullptr;
   int32_t* src = nullptr;
+  int32_t* chunk_counts = nullptr;  // [ceil(T_max/128)][E] per-chunk expert counts
+  int32_t* chunk_base = nullptr;    // [ceil(T_max/128)][E] first row of each (chunk, expert)
   int32_t* grp_rows = nullptr;
   int32_t* grp_base = nullptr;
   int32_t* ub1 = nullptr;
@@ -72,7 +72,8 @@ struct afd_ffn_handle {
   void* hin = nullptr;       // [T_max][H] bf16 staging for afd_ffn_forward_host
   void* hout = nullptr;
 
-  CUtensorMap tm_w13, tm_w2, tm_xp, tm_act;
+  CUtensorMap tm_w13, tm_w2, tm_wr;
+  CUtensorMap tm_xp[2], tm_act[2];  // token rows for the [narrow, wide] shapes (box heights differ)
   cudaStream_t last_stream = nullptr;
   int last_cuda_error = 0;
   cudaEvent_t events[AFD_FFN_NUM_STAGES + 1];
@@ -150,35 +151,97 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, STAGES, FP8, MODE, SPLIT>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, STAGES, SPLIT>());
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, ST, SPLIT, MODE>());
 }
 
-// (gate/up, down) kernel pairs of each path and tile shape
+// (gate/up, down) kernel pairs of each path and tile shape: N tile and ring stages of each
+// GEMM.  Compile-time tunable for tile sweeps: -DAFD_<path>_BN=.. -DAFD_<path>_ST=..
+// bf16 decode, gate/up
+#ifndef AFD_NB_G1_BN
+#define AFD_NB_G1_BN 32
+#endif
+#ifndef AFD_NB_G1_ST
+#define AFD_NB_G1_ST 6
+#endif
+// bf16 decode, down (hi and lo activation rows in one MMA)
+#ifndef AFD_NB_G2_BN
+#define AFD_NB_G2_BN 32
+#endif
+#ifndef AFD_NB_G2_ST
+#define AFD_NB_G2_ST 5
+#endif
+// bf16 large micro-batch, gate/up
+#ifndef AFD_WB_G1_BN
+#define AFD_WB_G1_BN 128
+#endif
+#ifndef AFD_WB_G1_ST
+#define AFD_WB_G1_ST 4
+#endif
+// bf16 large micro-batch, down (two activation planes per stage)
+#ifndef AFD_WB_G2_BN
+#define AFD_WB_G2_BN 128
+#endif
+#ifndef AFD_WB_G2_ST
+#define AFD_WB_G2_ST 3
+#endif
+// W8A8 decode, gate/up
+#ifndef AFD_NF_G1_BN
+#define AFD_NF_G1_BN 32
+#endif
+#ifndef AFD_NF_G1_ST
+#define AFD_NF_G1_ST 6
+#endif
+// W8A8 decode, down
+#ifndef AFD_NF_G2_BN
+#define AFD_NF_G2_BN 32
+#endif
+#ifndef AFD_NF_G2_ST
+#define AFD_NF_G2_ST 6
+#endif
+// W8A8 large micro-batch, gate/up
+#ifndef AFD_WF_G1_BN
+#define AFD_WF_G1_BN 128
+#endif
+#ifndef AFD_WF_G1_ST
+#define AFD_WF_G1_ST 4
+#endif
+// W8A8 large micro-batch, down
+#ifndef AFD_WF_G2_BN
+#define AFD_WF_G2_BN 128
+#endif
+#ifndef AFD_WF_G2_ST
+#define AFD_WF_G2_ST 4
+#endif
+
+template <int BN1, int ST1, int BN2, int ST2, bool SPLIT>
+struct GemmPairT {
+  static constexpr int bn1 = BN1, st1 = ST1, bn2 = BN2, st2 = ST2;
+  static constexpr bool split = SPLIT;
+};
 template <bool FP8, bool NARROW>
 struct GemmPair;
 template <>
-struct GemmPair<false, true> {  // bf16 decode
-  static constexpr int bn1 = kNarrowBN, st1 = kNarrowStages, bn2 = kNarrowBN, st2 = kNarrowSplitStages;
-  static constexpr bool split = true;
-};
+struct GemmPair<false, true> : GemmPairT<AFD_NB_G1_BN, AFD_NB_G1_ST, AFD_NB_G2_BN, AFD_NB_G2_ST, true> {};
 template <>
-struct GemmPair<false, false> {  // bf16 large micro-batch
-  static constexpr int bn1 = kWideBN, st1 = kWideStages, bn2 = kWideSplitBN, st2 = kWideStages;
-  static constexpr bool split = true;
-};
+struct GemmPair<false, false> : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true> {};
 template <>
-struct GemmPair<true, true> {  // W8A8 decode
-  static constexpr int bn1 = kNarrowBN, st1 = kNarrowStages, bn2 = kNarrowBN, st2 = kNarrowStages;
-  static constexpr bool split = false;
-};
+struct GemmPair<true, true> : GemmPairT<AFD_NF_G1_BN, AFD_NF_G1_ST, AFD_NF_G2_BN, AFD_NF_G2_ST, false> {};
 template <>
-struct GemmPair<true, false> {  // W8A8 large micro-batch
-  static constexpr int bn1 = kWideBN, st1 = kWideStages, bn2 = kWideBN, st2 = kWideStages;
-  static constexpr bool split = false;
-};
+struct GemmPair<true, false> : GemmPairT<AFD_WF_G1_BN, AFD_WF_G1_ST, AFD_WF_G2_BN, AFD_WF_G2_ST, false> {};
+
+// Token-tile TMA box height of the gate/up (gemm = 1) or down (gemm = 2) kernel of a shape.
+template <bool NARROW>
+uint32_t box_rows(bool fp8, int gemm) {
+  if (fp8) {
+    using P = GemmPair<true, NARROW>;
+    return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, false, 1>::kBoxRows;
+  }
+  using P = GemmPair<false, NARROW>;
+  return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, P::split, 1>::kBoxRows;
+}
 
 template <bool FP8, bool NARROW>
 cudaError_t set_pair_attrs() {
@@ -192,14 +255,23 @@ template <bool FP8>
 cudaError_t set_all_gemm_attrs() {
   cudaError_t e = set_pair_attrs<FP8, true>();
   if (e != cudaSuccess) return e;
+  e = set_gemm_attr<kRouterBN, kRouterStages, false, 2, false>();
+  if (e != cudaSuccess) return e;
   return set_pair_attrs<FP8, false>();
 }
 
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT>
-void launch_gemm(const afd_ffn_handle* h, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args,
-                 cudaStream_t s) {
-  grouped_gemm_kernel<BN, STAGES, FP8, MODE, SPLIT>
-      <<<h->num_sms, 192, gemm_smem_bytes<BN, STAGES, SPLIT>(), s>>>(a, b, args);
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
+void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
+  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, 192, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, args);
+}
+
+// K split of the tensor-core router: enough units to cover the SMs, every split non-empty.
+void router_ksplit(int T, int H, int E, int sms, int* ksplit, int* kc_per) {
+  const int kchunks = H / 64;
+  const int base = ((T + kRouterBN - 1) / kRouterBN) * ((E + 127) / 128);
+  const int want = std::max(1, std::min(kchunks, (sms + base - 1) / base));
+  *kc_per = (kchunks + want - 1) / want;
+  *ksplit = (kchunks + *kc_per - 1) / *kc_per;
 }
 
 void record(afd_ffn_handle* h, int stage, cudaStream_t s) {
@@ -208,17 +280,34 @@ void record(afd_ffn_handle* h, int stage, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------ stages
+// Router on the tensor cores (grouped GEMM, MODE 2): logits [T][E] fp32 into h->part, then the
+// warp-per-token top-k.  The hidden states' TMA descriptor is encoded per call (host only).
 int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float* w, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
-  int nsplit = 1, per = 1;
-  router_split(T, c.H, c.E, h->num_sms, &nsplit, &per);
+  CUtensorMap tm_h;
+  if (!encode_2d(&tm_h, hidden, false, c.H, static_cast<uint64_t>(T), GemmShape<kRouterBN, false, 2>::kBoxRows))
+    return AFD_ERR_INVALID_ARG;
+  int ksplit = 1, kc_per = 1;
+  router_ksplit(T, c.H, c.E, h->num_sms, &ksplit, &kc_per);
+  GemmArgs a{};
+  a.G = 1;
+  a.single_rows = T;
+  a.single_mt = (c.E + 127) / 128;
+  a.single_total = ((T + kRouterBN - 1) / kRouterBN) * a.single_mt * ksplit;
+  a.kc_per = kc_per;
+  a.K = c.H;
+  a.a_rows = c.E;
+  a.mt_stride = 128;
+  a.second_off = c.E;  // plane stride of the [3][E][H] weights
+  a.out = h->part;
+  a.out_ld = c.E;
+  a.err = h->err;
   record(h, 0, s);
-  dim3 grid((c.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
-  router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, h->part, T,
-                                            c.H, c.E, per);
+  launch_gemm<kRouterBN, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
   record(h, 1, s);
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, nsplit, c.has_router_bias ? h->w.router_bias : nullptr, T,
-                                                 c.E, c.k, idx, w);
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, c.has_router_bias ? h->w.router_bias : nullptr, T,
+                                                 c.E, c.k, idx, w, static_cast<const __nv_bfloat16*>(hidden),
+                                                 h->w.router_w, c.H);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -226,15 +315,18 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
 int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T, int32_t* counts, int32_t* offsets,
                 int32_t* pos, int32_t* src, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
+  const int nchunks = (T + kChunkTokens - 1) / kChunkTokens;
   record(h, 2, s);
-  dispatch_order_kernel<<<1, kDispatchThreads, 0, s>>>(idx, T, c.k, c.E, counts, offsets, pos, src, h->err);
+  dispatch_count_kernel<<<nchunks, kCountThreads, 0, s>>>(idx, T, c.k, c.E, pos, h->chunk_counts, h->err);
+  dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(h->chunk_counts, nchunks, c.E, counts, offsets, h->chunk_base);
   record(h, 3, s);
+  const __nv_bfloat16* hb = static_cast<const __nv_bfloat16*>(hidden);
   if (h->fp8)
-    gather_rows_kernel<true><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), pos, T, c.k, c.H, T * c.k,
-                                               c.n_shared, T * c.k, h->xp, h->xscale, h->err);
+    gather_rows_kernel<true><<<T, 256, 0, s>>>(hb, idx, h->chunk_base, pos, src, T, c.k, c.E, c.H, c.n_shared,
+                                               h->xp, h->xscale);
   else
-    gather_rows_kernel<false><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), pos, T, c.k, c.H,
-                                                T * c.k, c.n_shared, T * c.k, h->xp, h->xscale, h->err);
+    gather_rows_kernel<false><<<T, 256, 0, s>>>(hb, idx, h->chunk_base, pos, src, T, c.k, c.E, c.H, c.n_shared,
+                                                h->xp, h->xscale);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -242,9 +334,11 @@ int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T
 template <bool FP8, bool NARROW>
 void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   using P = GemmPair<FP8, NARROW>;
+  const int shape = NARROW ? 0 : 1;
   const afd_ffn_cfg& c = h->cfg;
   const int R = T * c.k + T;
   GemmArgs g1{};
+  g1.single_rows = -1;  // grouped: units come from the device schedule
   g1.grp_rows = h->grp_rows;
   g1.grp_base = h->grp_base;
   g1.unit_base = h->ub1;
@@ -256,13 +350,16 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g1.out = h->act;
   g1.out_ld = c.I;
   g1.lo_rows = h->R_max;
+  // decode streams each weight tile once; large micro-batches share it between N tiles
+  g1.a_policy = NARROW ? kEvictFirst : kEvictNormal;
   g1.a_scale = h->w.w13_scale;
   g1.b_scale = h->xscale;
   g1.err = h->err;
   record(h, 5, s);
-  launch_gemm<P::bn1, P::st1, FP8, 0, false>(h, h->tm_w13, h->tm_xp, g1, s);
+  launch_gemm<P::bn1, P::st1, FP8, 0, false>(h->num_sms, h->tm_w13, h->tm_xp[shape], g1, s);
   record(h, 6, s);
-  if (FP8) quantize_act_kernel<<<R, 256, 0, s>>>(static_cast<const float*>(h->act), c.I, h->actq, h->ascale);
+  if (FP8)
+    quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
   GemmArgs g2 = g1;
   g2.unit_base = h->ub2;
   g2.K = c.I;
@@ -274,7 +371,7 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g2.a_scale = h->w.w2_scale;
   g2.b_scale = h->ascale;
   record(h, 7, s);
-  launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(h, h->tm_w2, h->tm_act, g2, s);
+  launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(h->num_sms, h->tm_w2, h->tm_act[shape], g2, s);
 }
 
 int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
@@ -391,11 +488,11 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   h->R_max = cfg->T_max * (cfg->k + 1);
 
   const afd_ffn_cfg& c = h->cfg;
-  size_t part = 0;
+  size_t part = 0;  // partial router logits [ksplit][T][E], largest over T <= T_max
   for (int T = 1; T <= c.T_max; ++T) {
-    int ns, per;
-    router_split(T, c.H, c.E, sms, &ns, &per);
-    part = std::max(part, static_cast<size_t>(ns) * T * c.E);
+    int ks, per;
+    router_ksplit(T, c.H, c.E, sms, &ks, &per);
+    part = std::max(part, static_cast<size_t>(ks) * T * c.E);
   }
   h->part_floats = part;
 
@@ -407,10 +504,13 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
       {reinterpret_cast<void**>(&h->part), part * 4},
       {reinterpret_cast<void**>(&h->idx), Tm * c.k * 4},
       {reinterpret_cast<void**>(&h->wts), Tm * c.k * 4},
+      {&h->wr_planes, 3 * static_cast<size_t>(c.E) * c.H * 2},
       {reinterpret_cast<void**>(&h->counts), static_cast<size_t>(c.E) * 4},
       {reinterpret_cast<void**>(&h->offsets), static_cast<size_t>(c.E + 1) * 4},
       {reinterpret_cast<void**>(&h->pos), Tm * c.k * 4},
       {reinterpret_cast<void**>(&h->src), Tm * c.k * 4},
+      {reinterpret_cast<void**>(&h->chunk_counts), (Tm + kChunkTokens - 1) / kChunkTokens * c.E * 4},
+      {reinterpret_cast<void**>(&h->chunk_base), (Tm + kChunkTokens - 1) / kChunkTokens * c.E * 4},
       {reinterpret_cast<void**>(&h->grp_rows), static_cast<size_t>(h->G) * 4},
       {reinterpret_cast<void**>(&h->grp_base), static_cast<size_t>(h->G) * 4},
       {reinterpret_cast<void**>(&h->ub1), static_cast<size_t>(h->G + 1) * 4},
@@ -439,13 +539,25 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   h->act = act_p;
 
   const uint64_t G = h->G;
+  // token-row maps: box heights must match GemmShape<...>::kBoxRows of the kernels using them
+  const void* act_src = h->fp8 ? static_cast<const void*>(h->actq) : h->act;
+  const uint64_t act_rows = h->fp8 ? R : 2 * R;
+  const uint32_t box_xp[2] = {box_rows<true>(h->fp8, 1), box_rows<false>(h->fp8, 1)};
+  const uint32_t box_act[2] = {box_rows<true>(h->fp8, 2), box_rows<false>(h->fp8, 2)};
   bool ok = encode_2d(&h->tm_w13, weights->w13, h->fp8, c.H, G * 2 * c.I, 128) &&
             encode_2d(&h->tm_w2, weights->w2, h->fp8, c.I, G * c.H, 128) &&
-            encode_2d(&h->tm_xp, h->xp, h->fp8, c.H, R, 16) &&
-            encode_2d(&h->tm_act, h->fp8 ? static_cast<const void*>(h->actq) : h->act, h->fp8, c.I,
-                      h->fp8 ? R : 2 * R, 16);
+            encode_2d(&h->tm_xp[0], h->xp, h->fp8, c.H, R, box_xp[0]) &&
+            encode_2d(&h->tm_xp[1], h->xp, h->fp8, c.H, R, box_xp[1]) &&
+            encode_2d(&h->tm_act[0], act_src, h->fp8, c.I, act_rows, box_act[0]) &&
+            encode_2d(&h->tm_act[1], act_src, h->fp8, c.I, act_rows, box_act[1]) &&
+            encode_2d(&h->tm_wr, h->wr_planes, false, c.H, 3 * static_cast<uint64_t>(c.E), 128);
   if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
+  if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  router_split_planes_kernel<<<256, 256>>>(weights->router_w, static_cast<size_t>(c.E) * c.H,
+                                           static_cast<__nv_bfloat16*>(h->wr_planes));
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
   *out = h;
   return AFD_OK;
@@ -626,7 +738,8 @@ extern "C" int afd_ffn_route_static(const void* hidden, const float* router_w, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
   router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), router_w, part, T, H, E, per);
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w);
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w, nullptr,
+                                                 nullptr, H);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;

@@ -5,6 +5,8 @@
 // GPUs it is an all-to-all, here a local permutation).  Order taken: expert-major, and inside
 // an expert ascending token index, so every expert's rows are one contiguous block:
 //   counts[e], offsets = exclusive prefix sum, pos[t,j] = offsets[e] + #{t' < t chose e}.
+// Three launches: per-chunk ranks and counts (many CTAs), a scan over chunks and experts
+// (one CTA), and the final positions fused with the row gather (one CTA per token).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -14,27 +16,27 @@
 
 namespace afd {
 
-constexpr int kDispatchThreads = 1024;
 constexpr int kMaxExperts = 256;
+constexpr int kChunkTokens = 128;   // tokens per CTA of dispatch_count_kernel
+constexpr int kCountThreads = 256;  // 8 warps
 
-// One CTA of 1024 threads.  Each warp takes one contiguous segment of the flat (t, j) array
-// (flat order = token order for any one expert, since a token selects an expert at most once),
-// ranks its pairs per expert 32 at a time with a warp match (stable inside the segment) and
-// counts them per expert; the per-warp counts are then prefix-summed across warps and experts
-// and a second pass turns local ranks into global positions.  No atomics on the data path.
-__global__ void __launch_bounds__(kDispatchThreads)
-dispatch_order_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
-                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                      int32_t* __restrict__ pos, int32_t* __restrict__ src, int* err) {
-  __shared__ int cnt[32][kMaxExperts];
-  __shared__ int ebase[kMaxExperts];
+// Dispatch order, step 1 of 3 (many CTAs).  CTA c takes the tokens [c*128, (c+1)*128) and ranks
+// their (t, j) pairs per expert in flat order (flat order = token order for any one expert,
+// since a token selects an expert at most once): each warp ranks a contiguous part 32 pairs at
+// a time with a warp match, then the warps' counts are prefix-summed per expert.  Writes the
+// rank inside the chunk to pos[t, j] (-1 for an expert outside [0, E): flagged, skipped) and
+// the chunk's per-expert counts to chunk_counts[c][E].  No atomics on the data path.
+__global__ void __launch_bounds__(kCountThreads)
+dispatch_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __restrict__ pos,
+                      int32_t* __restrict__ chunk_counts, int* err) {
+  __shared__ int cnt[kCountThreads / 32][kMaxExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 32 * kMaxExperts; i += kDispatchThreads) (&cnt[0][0])[i] = 0;
+  for (int i = tid; i < (kCountThreads / 32) * kMaxExperts; i += kCountThreads) (&cnt[0][0])[i] = 0;
   __syncthreads();
-
-  const int n = T * k;
-  const int seg = ((n + 31) / 32 + 31) & ~31;
-  const int begin = min(n, warp * seg), end = min(n, begin + seg);
+  const int p0 = blockIdx.x * kChunkTokens * k;
+  const int p1 = min(T, (blockIdx.x + 1) * kChunkTokens) * k;
+  const int seg = (((p1 - p0) + 7) / 8 + 31) & ~31;
+  const int begin = min(p1, p0 + warp * seg), end = min(p1, begin + seg);
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int b = begin; b < end; b += 32) {
     const int i = b + lane;
@@ -48,7 +50,7 @@ dispatch_order_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
     const int before = valid ? cnt[warp][e] : 0;
     __syncwarp();
     if (valid) {
-      pos[i] = before + rank;                       // local rank, finished below
+      pos[i] = before + rank;
       if (rank == 0) cnt[warp][e] = before + __popc(grp);
     } else if (in) {
       pos[i] = -1;
@@ -56,76 +58,99 @@ dispatch_order_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
     __syncwarp();
   }
   __syncthreads();
-  if (tid < E) {  // exclusive prefix over warps, per expert
+  if (tid < E) {  // exclusive prefix over the warps, per expert; the total is the chunk's count
     int run = 0;
-    for (int w = 0; w < 32; ++w) {
+#pragma unroll
+    for (int w = 0; w < kCountThreads / 32; ++w) {
       const int c = cnt[w][tid];
       cnt[w][tid] = run;
       run += c;
     }
-    ebase[tid] = run;
-    counts[tid] = run;
-  }
-  __syncthreads();
-  if (warp == 0) {  // exclusive prefix over experts, 8 per lane
-    int v[8], s = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      v[i] = e < E ? ebase[e] : 0;
-      s += v[i];
-    }
-    const int incl = warp_incl_scan(s, lane);
-    int run = incl - s;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      if (e < E) { ebase[e] = run; offsets[e] = run; }
-      run += v[i];
-    }
-    if (lane == 31) offsets[E] = incl;
+    chunk_counts[static_cast<size_t>(blockIdx.x) * E + tid] = run;
   }
   __syncthreads();
   for (int b = begin; b < end; b += 32) {
     const int i = b + lane;
     if (i >= end) continue;
     const int e = idx[i];
-    if (e < 0 || e >= E) continue;
-    const int p = ebase[e] + cnt[warp][e] + pos[i];
-    pos[i] = p;
-    src[p] = i / k;
+    if (e >= 0 && e < E) pos[i] += cnt[warp][e];
   }
 }
 
-// Row gather: dispatched row pos[t,j] <- hidden row t, and (shared expert) row shared_base + t
-// <- hidden row t.  bf16 rows are copied with 16-byte vectors.  W8A8: the row is quantised
-// first -- scale = amax / 448 (1 for a zero row), e4m3 = round-to-nearest-even, saturating,
-// of the fp32 quotient x / scale -- and the scale travels with every copy.
+// Dispatch order, step 2 of 3 (one CTA, thread e = expert e): counts[e] = sum over chunks,
+// offsets = exclusive prefix sum over experts (offsets[E] = valid pairs), and
+// chunk_base[c][e] = offsets[e] + rows of expert e in the chunks before c.
+__global__ void __launch_bounds__(kMaxExperts)
+dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E, int32_t* __restrict__ counts,
+                     int32_t* __restrict__ offsets, int32_t* __restrict__ chunk_base) {
+  __shared__ int wsum[kMaxExperts / 32];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = chunk_counts[static_cast<size_t>(c) * E + e];
+      chunk_base[static_cast<size_t>(c) * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+  }
+  const int incl = warp_incl_scan(run, lane);
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kMaxExperts / 32 ? wsum[lane] : 0;
+    const int iv = warp_incl_scan(v, lane);
+    if (lane < kMaxExperts / 32) wsum[lane] = iv - v;
+  }
+  __syncthreads();
+  const int excl = wsum[warp] + incl - run;
+  if (e < E) {
+    offsets[e] = excl;
+    for (int c = 0; c < nchunks; ++c) chunk_base[static_cast<size_t>(c) * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = excl + run;
+}
+
+// Dispatch order, step 3 of 3, fused with the row gather (one CTA per token t): the final
+// position of pair (t, j) is chunk_base[t / 128][e] + its rank inside the chunk; pos and src
+// are written, and hidden row t is copied to every dispatched row and (shared expert) to row
+// T*k + t.  bf16 rows move as 16-byte vectors.  W8A8: the row is quantised first --
+// scale = amax / 448 (1 for a zero row), e4m3 = round-to-nearest-even, saturating, of the fp32
+// quotient x / scale -- and the scale travels with every copy.
 template <bool FP8>
 __global__ void __launch_bounds__(256)
-gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __restrict__ pos,
-                   int T, int k, int H, int shared_base, int with_shared, int n_rows,
-                   uint8_t* __restrict__ xp, float* __restrict__ xscale, int* err) {
+gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __restrict__ idx,
+                   const int32_t* __restrict__ chunk_base, int32_t* __restrict__ pos,
+                   int32_t* __restrict__ src, int T, int k, int E, int H, int with_shared,
+                   uint8_t* __restrict__ xp, float* __restrict__ xscale) {
   __shared__ int dst[34];  // up to 32 routed + 1 shared destinations; count in [33]
   __shared__ float red[8];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    int nd = 0;
-    for (int j = 0; j < k; ++j) {
-      const int p = pos[static_cast<size_t>(t) * k + j];
-      if (p < 0) continue;
-      if (p >= n_rows) { atomicOr(err, kErrBadPos); continue; }
-      dst[nd++] = p;
+  if (tid < 32) {
+    int p = -1;
+    if (tid < k) {
+      const size_t ij = static_cast<size_t>(t) * k + tid;
+      const int e = idx[ij];
+      if (e >= 0 && e < E) {
+        p = chunk_base[static_cast<size_t>(t / kChunkTokens) * E + e] + pos[ij];
+        pos[ij] = p;
+        src[p] = t;
+      }
     }
-    if (with_shared) dst[nd++] = shared_base + t;
-    dst[33] = nd;
+    const unsigned m = __ballot_sync(0xffffffffu, p >= 0);
+    if (p >= 0) dst[__popc(m & ((1u << tid) - 1u))] = p;
+    if (tid == 0) {
+      int nd = __popc(m);
+      if (with_shared) dst[nd++] = T * k + t;
+      dst[33] = nd;
+    }
   }
   __syncthreads();
   const int nd = dst[33];
   const __nv_bfloat16* row = hidden + static_cast<size_t>(t) * H;
+  const uint4* s4 = reinterpret_cast<const uint4*>(row);
   if constexpr (!FP8) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(row);
     for (int v = tid; v < H / 8; v += blockDim.x) {
       const uint4 x = s4[v];
       for (int d = 0; d < nd; ++d)
@@ -133,65 +158,74 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __re
     }
   } else {
     float amax = 0.f;
-    for (int i = tid; i < H; i += blockDim.x) amax = fmaxf(amax, fabsf(__bfloat162float(row[i])));
+    for (int v = tid; v < H / 8; v += blockDim.x) {
+      const uint4 x = s4[v];
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
     amax = warp_max(amax);
     if ((tid & 31) == 0) red[tid >> 5] = amax;
     __syncthreads();
     if (tid < 32) {
-      float m = tid < (blockDim.x >> 5) ? red[tid] : 0.f;
-      m = warp_max(m);
-      if (tid == 0) red[0] = m;
+      float mx = tid < (blockDim.x >> 5) ? red[tid] : 0.f;
+      mx = warp_max(mx);
+      if (tid == 0) red[0] = mx;
     }
     __syncthreads();
     amax = red[0];
     const float scale = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
-    for (int v = tid; v < H / 4; v += blockDim.x) {
-      uint32_t packed = 0;
+    for (int v = tid; v < H / 8; v += blockDim.x) {  // the row is L1-resident by now
+      const uint4 x = s4[v];
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&x);
+      uint32_t q[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float x = __fdiv_rn(__bfloat162float(row[v * 4 + i]), scale);
-        packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3)) << (8 * i);
+        const float2 f = __bfloat1622float2(b[i]);
+        const uint32_t lo = __nv_cvt_float_to_fp8(__fdiv_rn(f.x, scale), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float_to_fp8(__fdiv_rn(f.y, scale), __NV_SATFINITE, __NV_E4M3);
+        q[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
       }
+      const uint2 packed = make_uint2(q[0], q[1]);
       for (int d = 0; d < nd; ++d)
-        reinterpret_cast<uint32_t*>(xp + static_cast<size_t>(dst[d]) * H)[v] = packed;
+        reinterpret_cast<uint2*>(xp + static_cast<size_t>(dst[d]) * H)[v] = packed;
     }
     if (tid < nd) xscale[dst[tid]] = scale;
   }
 }
 
-// W8A8: quantise each row of the fp32 SwiGLU output act32 [R][I] to e4m3 with its own
-// scale, the same rule as the hidden rows.  One CTA per row.
+// W8A8: quantise each row of the fp32 SwiGLU output act32 [R][I] to e4m3 with its own scale,
+// the same rule as the hidden rows.  One warp per row, eight rows per CTA; the second pass over
+// a row reads it from L1.
 __global__ void __launch_bounds__(256)
-quantize_act_kernel(const float* __restrict__ act32, int I, uint8_t* __restrict__ actq,
+quantize_act_kernel(const float* __restrict__ act32, int R, int I, uint8_t* __restrict__ actq,
                     float* __restrict__ ascale) {
-  __shared__ float red[8];
-  const size_t r = blockIdx.x;
-  const float* row = act32 + r * I;
-  const int tid = threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const size_t r = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= static_cast<size_t>(R)) return;
+  const float4* row = reinterpret_cast<const float4*>(act32 + r * I);
   float amax = 0.f;
-  for (int i = tid; i < I; i += blockDim.x) amax = fmaxf(amax, fabsf(row[i]));
-  amax = warp_max(amax);
-  if ((tid & 31) == 0) red[tid >> 5] = amax;
-  __syncthreads();
-  if (tid < 32) {
-    float m = tid < (blockDim.x >> 5) ? red[tid] : 0.f;
-    m = warp_max(m);
-    if (tid == 0) red[0] = m;
+  for (int v = lane; v < I / 4; v += 32) {
+    const float4 x = row[v];
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
   }
-  __syncthreads();
-  amax = red[0];
+  amax = warp_max(amax);
   const float scale = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
-  for (int v = tid; v < I / 4; v += blockDim.x) {
-    const float4 x = reinterpret_cast<const float4*>(row)[v];
+  uint32_t* out = reinterpret_cast<uint32_t*>(actq + r * I);
+  for (int v = lane; v < I / 4; v += 32) {
+    const float4 x = row[v];
     const float xv[4] = {x.x, x.y, x.z, x.w};
     uint32_t packed = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(xv[i], scale), __NV_SATFINITE, __NV_E4M3))
                 << (8 * i);
-    reinterpret_cast<uint32_t*>(actq + r * I)[v] = packed;
+    out[v] = packed;
   }
-  if (tid == 0) ascale[r] = scale;
+  if (lane == 0) ascale[r] = scale;
 }
 
 // GEMM schedule from the group offsets: group g < E is expert g (rows offsets[g]..offsets[g+1]),

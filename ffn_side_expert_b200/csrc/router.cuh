@@ -9,6 +9,8 @@
 // router_logits_kernel: fp32 FMA GEMM, 64 tokens x 64 experts per CTA, 4x4 outputs per
 // thread, K tiles of 32 staged in shared memory, optionally split over K into partial sums
 // (deterministic: the top-k kernel adds the partials in split order).
+// (The tensor-core router used by afd_ffn_route / afd_ffn_forward is MODE 2 of the grouped GEMM
+// in gemm.cuh; router_logits_kernel serves the allocation-free afd_ffn_route_static.)
 // router_topk_kernel: one warp per token; the logits of E <= 256 experts sit 8 per lane,
 // k rounds of warp arg-max reductions pick the experts, a warp sum normalises the weights.
 #pragma once
@@ -88,9 +90,14 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __re
 }
 
 // One warp per token.  part: [nsplit][T][E] partial logits; bias: [E] or nullptr.
+// Selection uses the partial-sum logits.  With `hidden` and `wr` given (the tensor-core router,
+// whose fp32 accumulation is a few bits short of an fp32 FMA chain), the k selected logits are
+// then recomputed as fp32 FMA dot products -- each lane takes 8 consecutive hidden values per
+// step, the warp adds the lane sums -- and the gate weights come from those.
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __restrict__ bias,
-                   int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w) {
+                   int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w,
+                   const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr, int H) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -129,12 +136,64 @@ router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __re
     if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == j) { my_e = (be == 0x7fffffff) ? -1 : be; my_v = bv; }
   }
+  if (hidden != nullptr) {
+    // the k dot products are interleaved so that each lane keeps up to 8 loads in flight
+    const uint4* hr = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H);
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int ej[8];
+      float acc[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        ej[jj] = (j0 + jj < k) ? __shfl_sync(0xffffffffu, my_e, j0 + jj) : -1;
+        acc[jj] = 0.f;
+      }
+      for (int c = lane; c < H / 8; c += 32) {
+        const uint4 hv = hr[c];
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hv);
+        const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
+        const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          if (ej[jj] < 0) continue;
+          const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(ej[jj]) * H);
+          const float4 w0 = wrow[2 * c], w1 = wrow[2 * c + 1];
+          float a = acc[jj];
+          a = fmaf(f0.x, w0.x, a); a = fmaf(f0.y, w0.y, a); a = fmaf(f1.x, w0.z, a); a = fmaf(f1.y, w0.w, a);
+          a = fmaf(f2.x, w1.x, a); a = fmaf(f2.y, w1.y, a); a = fmaf(f3.x, w1.z, a); a = fmaf(f3.y, w1.w, a);
+          acc[jj] = a;
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const float sum = warp_sum(acc[jj]);
+        if (lane == j0 + jj && ej[jj] >= 0) my_v = bias ? sum + bias[ej[jj]] : sum;
+      }
+    }
+  }
   const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
   const float z = (lane < k) ? expf(my_v - vmax) : 0.f;
   const float sum = warp_sum(z);
   if (lane < k) {
     idx[static_cast<size_t>(t) * k + lane] = my_e;
     w[static_cast<size_t>(t) * k + lane] = z / sum;
+  }
+}
+
+// Router weights for the tensor-core router: Wr (fp32) -> three bf16 planes [3][n] with
+// hi = bf16(Wr), mid = bf16(Wr - hi), lo = bf16(Wr - hi - mid).  Both subtractions are exact in
+// fp32 (each plane holds the leading bits of what is left), so Wr = hi + mid + lo to ~2^-27.
+__global__ void router_split_planes_kernel(const float* __restrict__ wr, size_t n,
+                                           __nv_bfloat16* __restrict__ planes) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float w = wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    planes[i] = hi;
+    planes[n + i] = mid;
+    planes[2 * n + i] = __float2bfloat16_rn(r2);
   }
 }
 

@@ -155,8 +155,9 @@ const char *afd_ffn_strerror(int status);
  * and caps it (a stray cudaMalloc there fails or breaks the engine's accounting), and the
  * per-layer loop of an FFN service, where an allocation can synchronise the device in the
  * middle of a pipelined micro-batch.  afd_ffn_create allocates a workspace, so such callers
- * cannot use afd_ffn_route; this call computes the same thing (same kernels, same results
- * within the router's fp32 rounding; identical when T*E*splits fits, see below).
+ * cannot use afd_ffn_route; this call computes the same routing with the fp32 FMA router
+ * (afd_ffn_route runs the router on the tensor cores): the same experts, and gate weights
+ * equal to afd_ffn_route's up to the routers' fp32 rounding.
  *
  * Inputs (device, caller-owned, 16-byte aligned): hidden [T][H] bf16, router_w [E][H] fp32,
  * router_bias [E] fp32 or NULL.  Outputs: topk_idx [T][k] int32, topk_w [T][k] fp32.
@@ -165,7 +166,7 @@ const char *afd_ffn_strerror(int status);
  * AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS floats (4 MiB) that every GPU loading the library holds
  * until the process exits.  T*E must not exceed it; larger problems return
  * AFD_ERR_UNSUPPORTED before any device work (the split of the reduction over H is narrowed
- * to fit, so results can differ from afd_ffn_route in the last fp32 bits when it is).
+ * to fit when needed, which changes only the fp32 summation order).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress with
  * that device current); make that first call before any stream capture on the device.
  * Every call on a device shares the one array: calls that can overlap on the GPU (different

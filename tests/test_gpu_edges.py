@@ -31,6 +31,7 @@ def _check_layer(L, T, tol=BF16_TOL):
     idx, _ = L.route(T)
     assert np.array_equal(idx.cpu().numpy(), ref["idx"])
     err = rel_max_err(to64(out), ref["out"])
+    print(f"{L.cfg.name} T={T}: max|err|/RMS = {err:.4e} (bar {tol})")
     assert err <= tol, err
     return out
 
@@ -125,8 +126,8 @@ def test_all_experts_selected_with_shared_expert():
 
 
 def test_wide_tiles_with_several_n_tiles_per_expert():
-    # T*k > 32 E selects the wide tiles (N up to 256); 600 tokens over 2 experts gives each
-    # expert ~300 rows: two N tiles, the second ragged
+    # T*k > 32 E selects the wide tiles (N up to 128); 600 tokens over 2 experts gives each
+    # expert ~300 rows: several N tiles, the last one ragged
     cfg = synth.MoEConfig("wide", T=600, H=256, E=2, k=1, I=256, S=1, seed=24)
     L = Layer(cfg, redraws=_redraws(cfg))
     try:

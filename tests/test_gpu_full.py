@@ -62,6 +62,7 @@ def test_sampled_outputs_match_oracle(big):
     assert np.isfinite(got).all()
     tol = FP8_TOL if big.fp8 else BF16_TOL
     err = rel_max_err(got, ref["out"])
+    print(f"{big.cfg.name}: sampled tokens {len(tok)}, max|err|/RMS = {err:.4e} (bar {tol})")
     assert err <= tol, f"{big.cfg.name}: max|err|/RMS = {err:.3e}"
 
 

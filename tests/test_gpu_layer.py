@@ -71,6 +71,7 @@ def test_forward_and_staged_agree_with_oracle(layer):
     torch.cuda.synchronize()
     assert layer.mod.get_error() == 0
     err = rel_max_err(to64(out), ref["out"])
+    print(f"{layer.cfg.name}: max|err|/RMS = {err:.4e} (bar {BF16_TOL})")
     assert err <= BF16_TOL, err
     assert torch.equal(out, staged)                    # same kernels, same order
 
