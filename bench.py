@@ -295,7 +295,9 @@ def report_ours(args, world, r) -> dict:
     tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.dtype == "fp8" else 1.0)
     t_tc = acct["flops"] / (tc_peak * 1e12)
     t_roof = max(t_hbm, t_tc)
-    launches = 9 if cfg.dtype == "fp8" else 8
+    # router GEMM, top-k, refine, dispatch count, dispatch scan, gather, schedule, gate/up GEMM,
+    # (W8A8: activation quantisation), down GEMM, combine
+    launches = 11 if cfg.dtype == "fp8" else 10
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

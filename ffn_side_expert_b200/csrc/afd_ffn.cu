@@ -67,7 +67,7 @@ struct afd_ffn_handle {
   void* act = nullptr;       // [2][R_max][I] bf16 hi/lo planes (or [R_max][I] fp32 in W8A8)
   uint8_t* actq = nullptr;   // W8A8: [R_max][I] e4m3
   float* ascale = nullptr;   // W8A8: [R_max]
-  float* Y = nullptr;        // [R_max][H] fp32
+  float* Y = nullptr;        // [R_max][H] fp32 (bf16 on the W8A8 path)
   int* err = nullptr;        // device error word
   void* hin = nullptr;       // [T_max][H] bf16 staging for afd_ffn_forward_host
   void* hout = nullptr;
@@ -305,9 +305,10 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
   record(h, 0, s);
   launch_gemm<kRouterBN, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
   record(h, 1, s);
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, c.has_router_bias ? h->w.router_bias : nullptr, T,
-                                                 c.E, c.k, idx, w, static_cast<const __nv_bfloat16*>(hidden),
-                                                 h->w.router_w, c.H);
+  const float* bias = c.has_router_bias ? h->w.router_bias : nullptr;
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
+  router_refine_kernel<<<T, 32 * c.k, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, bias, c.H,
+                                             c.k, idx, w);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -402,8 +403,13 @@ int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream
 int run_combine(afd_ffn_handle* h, const float* w, const int32_t* pos, int T, void* out, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   record(h, 8, s);
-  combine_kernel<<<T, 256, 0, s>>>(h->Y, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
-                                   static_cast<__nv_bfloat16*>(out), h->err);
+  if (h->fp8)
+    combine_kernel<__nv_bfloat16><<<T, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->Y), w, pos, T, c.k,
+                                                    c.H, T * c.k, c.n_shared, static_cast<__nv_bfloat16*>(out),
+                                                    h->err);
+  else
+    combine_kernel<float><<<T, 256, 0, s>>>(h->Y, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
+                                            static_cast<__nv_bfloat16*>(out), h->err);
   record(h, 9, s);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
@@ -611,6 +617,13 @@ int afd_ffn_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int32_t T, fl
   h->last_stream = s;
   if ((st = run_expert_gemm(h, offsets, T, s)) != AFD_OK) return st;
   const size_t H = h->cfg.H, rk = static_cast<size_t>(T) * h->cfg.k;
+  if (h->fp8) {  // the W8A8 expert outputs are held as bf16: widen them on the way out
+    const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(h->Y);
+    if (Y) bf16_to_f32_kernel<<<4 * h->num_sms, 256, 0, s>>>(yb, Y, rk * H);
+    if (Ys) bf16_to_f32_kernel<<<4 * h->num_sms, 256, 0, s>>>(yb + rk * H, Ys, static_cast<size_t>(T) * H);
+    AFD_CUDA(h, cudaGetLastError());
+    return AFD_OK;
+  }
   if (Y) AFD_CUDA(h, cudaMemcpyAsync(Y, h->Y, rk * H * 4, cudaMemcpyDeviceToDevice, s));
   if (Ys) AFD_CUDA(h, cudaMemcpyAsync(Ys, h->Y + rk * H, static_cast<size_t>(T) * H * 4, cudaMemcpyDeviceToDevice, s));
   return AFD_OK;
@@ -738,8 +751,7 @@ extern "C" int afd_ffn_route_static(const void* hidden, const float* router_w, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
   router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), router_w, part, T, H, E, per);
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w, nullptr,
-                                                 nullptr, H);
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;

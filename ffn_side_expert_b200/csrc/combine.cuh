@@ -3,7 +3,8 @@
 // Combine returns the experts' outputs to their tokens (A/F 分离, 机制; an all-to-all
 // across GPUs, a gather here).  Reading taken: out[t] = sum_j w[t,j] * Y[pos[t,j]] + Ys[t],
 // summed in fp32 in j order with the shared expert last, rounded once to bf16.  No atomics:
-// one CTA per token, so the result does not depend on scheduling.
+// one CTA per token, so the result does not depend on scheduling.  Y is fp32 on the bf16 path
+// and bf16 on the W8A8 path (its 6e-2 error budget leaves room; it halves the bytes read).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -12,8 +13,17 @@
 
 namespace afd {
 
+__device__ __forceinline__ float4 load4(const float* p, size_t i) { return reinterpret_cast<const float4*>(p)[i]; }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p, size_t i) {
+  const uint2 u = reinterpret_cast<const uint2*>(p)[i];
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <typename YT>
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ Y, const float* __restrict__ w, const int32_t* __restrict__ pos,
+combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int32_t* __restrict__ pos,
                int T, int k, int H, int n_rows, int with_shared, __nv_bfloat16* __restrict__ out, int* err) {
   __shared__ int sp[32];
   __shared__ float sw[32];
@@ -25,21 +35,21 @@ combine_kernel(const float* __restrict__ Y, const float* __restrict__ w, const i
     sw[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
   }
   __syncthreads();
-  const float* ys = Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
+  const YT* ys = Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
   for (int v = threadIdx.x; v < H / 4; v += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const int p = sp[j];
       if (p < 0) continue;
       const float wj = sw[j];
-      const float4 y = reinterpret_cast<const float4*>(Y + static_cast<size_t>(p) * H)[v];
+      const float4 y = load4(Y + static_cast<size_t>(p) * H, v);
       acc.x = fmaf(wj, y.x, acc.x);
       acc.y = fmaf(wj, y.y, acc.y);
       acc.z = fmaf(wj, y.z, acc.z);
       acc.w = fmaf(wj, y.w, acc.w);
     }
     if (with_shared) {
-      const float4 s = reinterpret_cast<const float4*>(ys)[v];
+      const float4 s = load4(ys, v);
       acc.x += s.x; acc.y += s.y; acc.z += s.z; acc.w += s.w;
     }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
@@ -49,6 +59,13 @@ combine_kernel(const float* __restrict__ Y, const float* __restrict__ w, const i
     packed.y = *reinterpret_cast<uint32_t*>(&hi);
     reinterpret_cast<uint2*>(out + static_cast<size_t>(t) * H)[v] = packed;
   }
+}
+
+// Widen bf16 rows to fp32 (copy-out of the W8A8 expert outputs by afd_ffn_expert_gemm).
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[i] = __bfloat162float(src[i]);
 }
 
 }  // namespace afd

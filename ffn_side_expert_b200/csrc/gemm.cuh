@@ -56,7 +56,7 @@ struct GemmArgs {
   int a_rows;                // weight rows per group (2I gate/up, H down); router: valid rows E
   int mt_stride;             // weight rows between consecutive tile pairs (128 / 256)
   int second_off;            // offset of a pair's second tile (I / 128); router: plane stride E
-  void* out;                 // MODE 0: act (bf16 planes, or fp32 for W8A8); MODE 1: Y fp32;
+  void* out;                 // MODE 0: act (bf16 planes, or fp32 for W8A8); MODE 1: Y fp32 (bf16 for W8A8);
                              // MODE 2: partial logits fp32 [ksplit][rows][E]
   int out_ld;                // elements per output row
   int lo_rows;               // bf16 two-term activations: row offset of the lo plane (R_max)
@@ -388,6 +388,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                   o[row * args.out_ld + wrow0] = hi;
                   o[(static_cast<size_t>(args.lo_rows) + row) * args.out_ld + wrow0] = lo;
                 }
+              } else if constexpr (FP8) {  // W8A8: expert outputs kept as bf16 (combine input)
+                __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.out) + row * args.out_ld;
+                y[wrow0] = __float2bfloat16_rn(v0);
+                y[wrow1] = __float2bfloat16_rn(v1);
               } else {
                 float* y = static_cast<float*>(args.out) + row * args.out_ld;
                 y[wrow0] = v0;

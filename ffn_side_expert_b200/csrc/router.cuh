@@ -10,7 +10,8 @@
 // thread, K tiles of 32 staged in shared memory, optionally split over K into partial sums
 // (deterministic: the top-k kernel adds the partials in split order).
 // (The tensor-core router used by afd_ffn_route / afd_ffn_forward is MODE 2 of the grouped GEMM
-// in gemm.cuh; router_logits_kernel serves the allocation-free afd_ffn_route_static.)
+// in gemm.cuh followed by router_refine_kernel; router_logits_kernel serves the allocation-free
+// afd_ffn_route_static.)
 // router_topk_kernel: one warp per token; the logits of E <= 256 experts sit 8 per lane,
 // k rounds of warp arg-max reductions pick the experts, a warp sum normalises the weights.
 #pragma once
@@ -89,15 +90,12 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __re
   }
 }
 
-// One warp per token.  part: [nsplit][T][E] partial logits; bias: [E] or nullptr.
-// Selection uses the partial-sum logits.  With `hidden` and `wr` given (the tensor-core router,
-// whose fp32 accumulation is a few bits short of an fp32 FMA chain), the k selected logits are
-// then recomputed as fp32 FMA dot products -- each lane takes 8 consecutive hidden values per
-// step, the warp adds the lane sums -- and the gate weights come from those.
+// One warp per token.  part: [nsplit][T][E] partial logits (summed in split order); bias: [E]
+// or nullptr.  Writes the k selected experts (descending logit, ties to the lower index) and
+// the softmax of their logits.
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __restrict__ bias,
-                   int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w,
-                   const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr, int H) {
+                   int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -136,46 +134,57 @@ router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __re
     if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == j) { my_e = (be == 0x7fffffff) ? -1 : be; my_v = bv; }
   }
-  if (hidden != nullptr) {
-    // the k dot products are interleaved so that each lane keeps up to 8 loads in flight
-    const uint4* hr = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H);
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      int ej[8];
-      float acc[8];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        ej[jj] = (j0 + jj < k) ? __shfl_sync(0xffffffffu, my_e, j0 + jj) : -1;
-        acc[jj] = 0.f;
-      }
-      for (int c = lane; c < H / 8; c += 32) {
-        const uint4 hv = hr[c];
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hv);
-        const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
-        const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          if (ej[jj] < 0) continue;
-          const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(ej[jj]) * H);
-          const float4 w0 = wrow[2 * c], w1 = wrow[2 * c + 1];
-          float a = acc[jj];
-          a = fmaf(f0.x, w0.x, a); a = fmaf(f0.y, w0.y, a); a = fmaf(f1.x, w0.z, a); a = fmaf(f1.y, w0.w, a);
-          a = fmaf(f2.x, w1.x, a); a = fmaf(f2.y, w1.y, a); a = fmaf(f3.x, w1.z, a); a = fmaf(f3.y, w1.w, a);
-          acc[jj] = a;
-        }
-      }
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const float sum = warp_sum(acc[jj]);
-        if (lane == j0 + jj && ej[jj] >= 0) my_v = bias ? sum + bias[ej[jj]] : sum;
-      }
-    }
-  }
   const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
   const float z = (lane < k) ? expf(my_v - vmax) : 0.f;
   const float sum = warp_sum(z);
   if (lane < k) {
     idx[static_cast<size_t>(t) * k + lane] = my_e;
     w[static_cast<size_t>(t) * k + lane] = z / sum;
+  }
+}
+
+// Gate weights from exact fp32 logits of the selected experts.  The tensor-core router's fp32
+// accumulation over 3 x H terms is a few bits short of an fp32 FMA chain: good enough to select
+// (the selection margin is far larger), not for the weights.  One CTA per token, warp j
+// recomputes logit j = hidden[t] . Wr[idx[t][j]] (+ bias) with fp32 FMAs (each lane takes 8
+// consecutive hidden values per step, the warp adds the lane sums); warp 0 then writes the
+// softmax over the k logits.  blockDim = 32 * k.
+__global__ void __launch_bounds__(1024)
+router_refine_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr,
+                     const float* __restrict__ bias, int H, int k, const int32_t* __restrict__ idx,
+                     float* __restrict__ w) {
+  __shared__ float lg[32];
+  const int t = blockIdx.x;
+  const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = idx[static_cast<size_t>(t) * k + j];
+  float acc = 0.f;
+  if (e >= 0) {
+    const uint4* hr = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H);
+    const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
+#pragma unroll 4
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 hv = hr[c];
+      const float4 w0 = wrow[2 * c], w1 = wrow[2 * c + 1];
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hv);
+      float2 f;
+      f = __bfloat1622float2(b[0]); acc = fmaf(f.x, w0.x, acc); acc = fmaf(f.y, w0.y, acc);
+      f = __bfloat1622float2(b[1]); acc = fmaf(f.x, w0.z, acc); acc = fmaf(f.y, w0.w, acc);
+      f = __bfloat1622float2(b[2]); acc = fmaf(f.x, w1.x, acc); acc = fmaf(f.y, w1.y, acc);
+      f = __bfloat1622float2(b[3]); acc = fmaf(f.x, w1.z, acc); acc = fmaf(f.y, w1.w, acc);
+    }
+    acc = warp_sum(acc);
+    if (bias) acc += bias[e];
+  } else {
+    acc = -INFINITY;
+  }
+  if (lane == 0) lg[j] = acc;
+  __syncthreads();
+  if (j == 0) {
+    const float v = lane < k ? lg[lane] : -INFINITY;
+    const float vmax = __shfl_sync(0xffffffffu, v, 0);  // selection order: logit 0 is the largest
+    const float z = lane < k ? expf(v - vmax) : 0.f;
+    const float sum = warp_sum(z);
+    if (lane < k) w[static_cast<size_t>(t) * k + lane] = z / sum;
   }
 }
 

@@ -107,9 +107,9 @@ int afd_ffn_permute(afd_ffn_handle *h, const void *hidden, const int32_t *topk_i
                     int32_t *counts, int32_t *offsets, int32_t *pos, int32_t *src, void *stream);
 
 /* Expert FFNs on the rows dispatched by the last afd_ffn_permute of this handle, grouped by
- * `offsets` [E+1] (device).  Writes the handle's internal output rows; when non-NULL also
- * copies them out: Y [T*k][H] fp32 (row p = the output of dispatched row p, unweighted) and
- * Ys [T][H] fp32 (shared expert; must be NULL when n_shared == 0). */
+ * `offsets` [E+1] (device).  Writes the handle's internal output rows (fp32; bf16 on the W8A8
+ * path); when non-NULL also copies them out as fp32: Y [T*k][H] (row p = the output of
+ * dispatched row p, unweighted) and Ys [T][H] (shared expert; must be NULL when n_shared == 0). */
 int afd_ffn_expert_gemm(afd_ffn_handle *h, const int32_t *offsets, int32_t T,
                         float *Y, float *Ys, void *stream);
 
