@@ -59,6 +59,8 @@ _SIGNATURES = {
     "afd_ffn_combine": (ctypes.c_int, [_P, _P, _P, _I, _P, _P]),
     "afd_ffn_forward": (ctypes.c_int, [_P, _P, _I, _P, _P]),
     "afd_ffn_forward_host": (ctypes.c_int, [_P, _P, _I, _P, _P]),
+    "afd_ffn_forward_host_batches": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p),
+                                                    ctypes.POINTER(ctypes.c_void_p), _I, _I, _P]),
     "afd_ffn_set_stage_events": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "afd_ffn_get_error": (ctypes.c_int, [_P]),
     "afd_ffn_last_cuda_error": (ctypes.c_int, [_P]),
@@ -156,6 +158,14 @@ def afd_ffn_forward_host(h, hidden_host, T, out_host, stream=None) -> int:
     return _lib.afd_ffn_forward_host(h, _ptr(hidden_host), T, _ptr(out_host), _stream(stream))
 
 
+def afd_ffn_forward_host_batches(h, hidden_host_list, out_host_list, T, stream=None) -> int:
+    """hidden_host_list / out_host_list: sequences of pinned host tensors [T, H] bf16."""
+    n = len(hidden_host_list)
+    ins = (ctypes.c_void_p * max(n, 1))(*[_ptr(x) for x in hidden_host_list])
+    outs = (ctypes.c_void_p * max(n, 1))(*[_ptr(x) for x in out_host_list])
+    return _lib.afd_ffn_forward_host_batches(h, ins, outs, n, T, _stream(stream))
+
+
 def afd_ffn_set_stage_events(h, events) -> int:
     """events: sequence of torch.cuda.Event (AFD_FFN_NUM_STAGES + 1 of them) or None.
 
@@ -246,6 +256,11 @@ class AfdFfn:
     def forward_host(self, hidden_host, out_host, T=None, stream=None):
         T = hidden_host.shape[0] if T is None else T
         self._check(afd_ffn_forward_host(self.h, hidden_host, T, out_host, stream), "afd_ffn_forward_host")
+
+    def forward_host_batches(self, hidden_host_list, out_host_list, T=None, stream=None):
+        T = hidden_host_list[0].shape[0] if T is None else T
+        self._check(afd_ffn_forward_host_batches(self.h, hidden_host_list, out_host_list, T, stream),
+                    "afd_ffn_forward_host_batches")
 
     def set_stage_events(self, events):
         self._events = events          # keep the events alive while the library records them

@@ -71,6 +71,10 @@ struct afd_ffn_handle {
   int* err = nullptr;        // device error word
   void* hin = nullptr;       // [T_max][H] bf16 staging for afd_ffn_forward_host
   void* hout = nullptr;
+  void* hin2 = nullptr;      // second staging pair of afd_ffn_forward_host_batches
+  void* hout2 = nullptr;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;   // copy streams of the batch loop
+  cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
 
   CUtensorMap tm_w13, tm_w2, tm_wr;
   CUtensorMap tm_xp[2], tm_act[2];  // token rows for the [narrow, wide] shapes (box heights differ)
@@ -530,6 +534,8 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
       {reinterpret_cast<void**>(&h->err), 256},
       {&h->hin, Tm * c.H * 2},
       {&h->hout, Tm * c.H * 2},
+      {&h->hin2, Tm * c.H * 2},
+      {&h->hout2, Tm * c.H * 2},
   };
   size_t total = 0;
   for (auto& p : pieces) total += (p.bytes + 255) & ~size_t(255);
@@ -564,7 +570,14 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
                                            static_cast<__nv_bfloat16*>(h->wr_planes));
   e = cudaGetLastError();
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
+  }
+  if (e != cudaSuccess) { afd_ffn_destroy(h); return cuda_fail(nullptr, e); }
   *out = h;
   return AFD_OK;
 }
@@ -572,6 +585,13 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
 void afd_ffn_destroy(afd_ffn_handle* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_done[i]) cudaEventDestroy(h->ev_done[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+  }
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   cudaFree(h->ws);
   delete h;
 }
@@ -668,6 +688,41 @@ int afd_ffn_forward_host(afd_ffn_handle* h, const void* hidden_host, int32_t T, 
   AFD_CUDA(h, cudaMemcpyAsync(h->hin, hidden_host, bytes, cudaMemcpyHostToDevice, s));
   if ((st = afd_ffn_forward(h, h->hin, T, h->hout, stream)) != AFD_OK) return st;
   AFD_CUDA(h, cudaMemcpyAsync(out_host, h->hout, bytes, cudaMemcpyDeviceToHost, s));
+  AFD_CUDA(h, cudaStreamSynchronize(s));
+  return AFD_OK;
+}
+
+int afd_ffn_forward_host_batches(afd_ffn_handle* h, const void* const* hidden_host, void* const* out_host,
+                                 int32_t n_batches, int32_t T, void* stream) {
+  if (!h || n_batches < 0) return AFD_ERR_INVALID_ARG;
+  int st = check_T(h, T);
+  if (st != AFD_OK) return st;
+  if (T == 0 || n_batches == 0) return AFD_OK;
+  if (!hidden_host || !out_host) return AFD_ERR_INVALID_ARG;
+  for (int i = 0; i < n_batches; ++i)
+    if (!hidden_host[i] || !out_host[i]) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * h->cfg.H * 2;
+  void* din[2] = {h->hin, h->hin2};
+  void* dout[2] = {h->hout, h->hout2};
+  // batch i uses staging slot i % 2.  copy_in: H2D of batch i once the layer of batch i-2 has
+  // consumed the slot; compute: the layer of batch i once its input landed and the D2H of
+  // batch i-2 has drained the output slot; copy_out: D2H of batch i once its layer is done.
+  for (int i = 0; i < n_batches; ++i) {
+    const int b = i & 1;
+    if (i >= 2) AFD_CUDA(h, cudaStreamWaitEvent(h->copy_in, h->ev_done[b], 0));
+    AFD_CUDA(h, cudaMemcpyAsync(din[b], hidden_host[i], bytes, cudaMemcpyHostToDevice, h->copy_in));
+    AFD_CUDA(h, cudaEventRecord(h->ev_in[b], h->copy_in));
+    AFD_CUDA(h, cudaStreamWaitEvent(s, h->ev_in[b], 0));
+    if (i >= 2) AFD_CUDA(h, cudaStreamWaitEvent(s, h->ev_out[b], 0));
+    if ((st = afd_ffn_forward(h, din[b], T, dout[b], stream)) != AFD_OK) return st;
+    AFD_CUDA(h, cudaEventRecord(h->ev_done[b], s));
+    AFD_CUDA(h, cudaStreamWaitEvent(h->copy_out, h->ev_done[b], 0));
+    AFD_CUDA(h, cudaMemcpyAsync(out_host[i], dout[b], bytes, cudaMemcpyDeviceToHost, h->copy_out));
+    AFD_CUDA(h, cudaEventRecord(h->ev_out[b], h->copy_out));
+  }
+  AFD_CUDA(h, cudaStreamSynchronize(h->copy_out));
   AFD_CUDA(h, cudaStreamSynchronize(s));
   return AFD_OK;
 }

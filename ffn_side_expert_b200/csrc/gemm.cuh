@@ -81,11 +81,16 @@ struct GemmShape {
   static constexpr int kBStage = (SPLIT_B ? 2 : 1) * kBTile;
   static constexpr int kStageBytes = kAStage + kBStage;
   // two-term activations in one MMA (hi rows, then lo rows): the N of an MMA doubles
-  static constexpr bool kConcat = SPLIT_B && BN <= 64;
+#ifndef AFD_CONCAT_MAX_BN
+#define AFD_CONCAT_MAX_BN 64
+#endif
+  static constexpr bool kConcat = SPLIT_B && BN <= AFD_CONCAT_MAX_BN;
   // rows per TMA box of a token tile: few large boxes keep the single producer thread from
   // becoming the bottleneck; a box may overrun the unit's rows (the MMA reads only n16 rows)
   // except in the concatenated layout, where the lo rows follow the hi rows directly
-  static constexpr int kBoxRows = kConcat ? 16 : (BN < 64 ? BN : 64);
+  static constexpr int kBoxRows = kConcat ? (BN <= 32 ? 16 : 32) : (BN < 64 ? BN : 64);
+  // concatenated layout: hi rows padded to whole boxes, then the lo rows
+  __device__ static int npad(int n16) { return kConcat ? (n16 + kBoxRows - 1) / kBoxRows * kBoxRows : n16; }
   static constexpr int kUnitCols = kNDU * BN * (kConcat ? 2 : 1);  // TMEM columns of one unit
   static constexpr int kNacc = (2 * kUnitCols <= 512) ? 2 : 1;  // unit buffers in TMEM
   static constexpr int kColsUsed = kNacc * kUnitCols;
@@ -227,8 +232,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int ya = w.g * args.a_rows + w.mt * args.mt_stride;
       const int nbox = (w.n16 + S::kBoxRows - 1) / S::kBoxRows;  // token-tile boxes per plane
       const uint32_t tx = S::kAStage + (SPLIT_B ? 2u : 1u) * static_cast<uint32_t>(nbox * S::kBoxRows) * 128u;
-      // the lo activation rows follow the hi rows (decode shape) or sit one tile further
-      const uint32_t lo_off = S::kConcat ? static_cast<uint32_t>(w.n16) * 128u : S::kBTile;
+      // the lo activation rows follow the (padded) hi rows or sit one tile further
+      const uint32_t lo_off = S::kConcat ? static_cast<uint32_t>(S::npad(w.n16)) * 128u : S::kBTile;
       const uint64_t apol = MODE == 2 ? kEvictLast : args.a_policy;
       for (int kc = w.kc0; kc < w.kc1; ++kc) {
         if (!mbar_wait(empty + 8u * s, ph ^ 1u, abort_flag)) { ok = false; break; }
@@ -268,7 +273,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       const Unit w = decode_unit<BN>(args, sched, u, kchunks);
-      const uint32_t idesc = idesc_m128(S::kConcat ? 2 * w.n16 : w.n16, FP8);
+      const uint32_t idesc = idesc_m128(S::kConcat ? 2 * S::npad(w.n16) : w.n16, FP8);
       if (!mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d0 = tmem + static_cast<uint32_t>(acc * S::kUnitCols);
@@ -354,10 +359,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tmem_ld16(t0 + c, r0);
           tmem_ld16(t1 + c, r1);
           tmem_ld_wait(r0, r1);
-          if constexpr (S::kConcat) {  // add the lo-plane half (columns n16..2*n16) of each tile
+          if constexpr (S::kConcat) {  // add the lo-plane half (columns npad..) of each tile
             uint32_t l0[16], l1[16];
-            tmem_ld16(t0 + w.n16 + c, l0);
-            tmem_ld16(t1 + w.n16 + c, l1);
+            tmem_ld16(t0 + S::npad(w.n16) + c, l0);
+            tmem_ld16(t1 + S::npad(w.n16) + c, l1);
             tmem_ld_wait(l0, l1);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {

@@ -116,6 +116,20 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 template <bool kFp8>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
+#ifdef AFD_MMA_NOMASK
+  if constexpr (kFp8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem), "l"(adesc),
+        "l"(bdesc), "r"(idesc), "r"(accumulate));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem), "l"(adesc),
+        "l"(bdesc), "r"(idesc), "r"(accumulate));
+  }
+  return;
+#endif
   const uint32_t z = 0;  // disable-output-lane mask: all lanes written
   if constexpr (kFp8) {
     asm volatile(

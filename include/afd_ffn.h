@@ -128,6 +128,17 @@ int afd_ffn_forward(afd_ffn_handle *h, const void *hidden, int32_t T, void *out,
 int afd_ffn_forward_host(afd_ffn_handle *h, const void *hidden_host, int32_t T, void *out_host,
                          void *stream);
 
+/* The FFN service's loop over a sequence of micro-batches held in HOST memory: for batch i,
+ * hidden_host[i] [T][H] bf16 is copied to the device, the layer runs, and the result is copied
+ * to out_host[i] [T][H] bf16.  Copies run on two copy streams owned by the handle and overlap
+ * the layer of the neighbouring batches (double-buffered device staging), the micro-pipeline of
+ * an A/F split in which the period tends to max(compute, transfer) instead of their sum (A/F
+ * 分离 page, section 深入推导, 微流水).  Results equal afd_ffn_forward's bit for bit.  `stream`
+ * runs the layer; the call synchronises everything it enqueued before returning.  Pinned host
+ * buffers are required for the copies to overlap.  0 <= T <= T_max, n_batches >= 0. */
+int afd_ffn_forward_host_batches(afd_ffn_handle *h, const void *const *hidden_host,
+                                 void *const *out_host, int32_t n_batches, int32_t T, void *stream);
+
 /* Optional stage timing: n_events cudaEvent_t handles (owned by the caller) that
  * afd_ffn_forward records on its stream before each stage and after the last one.  Stages,
  * in order: router logits, top-k, dispatch order, row gather, GEMM schedule, gate/up GEMM,

@@ -92,6 +92,9 @@ CONFIGS = {
     # W8A8 prefill chunk
     "w8a8_8192": MoEConfig("w8a8_8192", T=8192, H=7168, E=256, k=8, I=2048, S=1,
                            dtype="fp8", seed=4),
+    # W8A8 decode micro-batch (the serving benchmark's precision at the decode shape)
+    "w8a8_256": MoEConfig("w8a8_256", T=256, H=7168, E=256, k=8, I=2048, S=1,
+                          dtype="fp8", seed=5),
 }
 
 

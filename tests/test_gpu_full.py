@@ -17,7 +17,7 @@ from oracle import moe
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["dsv3_256", "dsv3_4096", "w8a8_8192"])
+@pytest.fixture(scope="module", params=["dsv3_256", "dsv3_4096", "w8a8_8192", "w8a8_256"])
 def big(request):
     L = Layer(synth.CONFIGS[request.param])
     L.routing = L.oracle_routing()

@@ -90,6 +90,22 @@ def test_forward_host_buffers(layer):
     assert torch.equal(hout, out.cpu())
 
 
+def test_forward_host_batches_pipeline(layer):
+    # four different micro-batches through the FFN-service loop (copies overlapped with the
+    # layer on separate streams) give the same bits as one forward per batch
+    T = layer.hidden.shape[0]
+    g = torch.Generator().manual_seed(7)
+    batches = [layer.hidden[torch.randperm(T, generator=g)].contiguous().pin_memory() for _ in range(4)]
+    outs = [torch.empty_like(b).pin_memory() for b in batches]
+    layer.mod.forward_host_batches(batches, outs)
+    for b, o in zip(batches, outs):
+        want = torch.empty((T, layer.cfg.H), dtype=torch.bfloat16, device="cuda")
+        layer.mod.forward(b.cuda(), want)
+        torch.cuda.synchronize()
+        assert torch.equal(o, want.cpu())
+    assert layer.mod.get_error() == 0
+
+
 def test_cuda_graph_replay(layer):
     eager = layer.forward().clone()
     out = torch.empty_like(eager)
