@@ -62,6 +62,9 @@ struct afd_ffn_handle {
   int32_t* grp_base = nullptr;
   int32_t* ub1 = nullptr;
   int32_t* ub2 = nullptr;
+  int32_t* tile_base = nullptr;  // [G] first N tile of each group
+  int* tile_done = nullptr;      // [N tiles] act-tile counters of the fused expert kernel
+  int max_tiles = 0;
   uint8_t* xp = nullptr;     // dispatched rows [R_max][H] bf16 / e4m3
   float* xscale = nullptr;   // [R_max]
   void* act = nullptr;       // [2][R_max][I] bf16 hi/lo planes (or [R_max][I] fp32 in W8A8)
@@ -220,17 +223,35 @@ cudaError_t set_gemm_attr() {
 #define AFD_WF_G2_ST 4
 #endif
 
-template <int BN1, int ST1, int BN2, int ST2, bool SPLIT>
+// bf16 decode shape: the gate/up and down GEMMs run fused in one launch (MODE 3) with stf ring
+// stages (measured on B200 at T=256: 3.45 ms fused vs 3.49 ms as two launches).  The large
+// micro-batch shape stays two launches: sharing one ring with the down GEMM's 64 KB stages
+// leaves the gate/up side three stages instead of four, which cost 0.95 ms at T=4096.
+#ifndef AFD_FUSED
+#define AFD_FUSED 1
+#endif
+#ifndef AFD_NB_F_ST
+#define AFD_NB_F_ST 5
+#endif
+#ifndef AFD_WB_F_ST
+#define AFD_WB_F_ST 0
+#endif
+
+template <int BN1, int ST1, int BN2, int ST2, bool SPLIT, int STF = 0>
 struct GemmPairT {
   static constexpr int bn1 = BN1, st1 = ST1, bn2 = BN2, st2 = ST2;
+  static constexpr int stf = STF;
   static constexpr bool split = SPLIT;
+  static constexpr bool fused = STF > 0 && BN1 == BN2 && AFD_FUSED;
 };
 template <bool FP8, bool NARROW>
 struct GemmPair;
 template <>
-struct GemmPair<false, true> : GemmPairT<AFD_NB_G1_BN, AFD_NB_G1_ST, AFD_NB_G2_BN, AFD_NB_G2_ST, true> {};
+struct GemmPair<false, true>
+    : GemmPairT<AFD_NB_G1_BN, AFD_NB_G1_ST, AFD_NB_G2_BN, AFD_NB_G2_ST, true, AFD_NB_F_ST> {};
 template <>
-struct GemmPair<false, false> : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true> {};
+struct GemmPair<false, false>
+    : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true, AFD_WB_F_ST> {};
 template <>
 struct GemmPair<true, true> : GemmPairT<AFD_NF_G1_BN, AFD_NF_G1_ST, AFD_NF_G2_BN, AFD_NF_G2_ST, false> {};
 template <>
@@ -250,9 +271,13 @@ uint32_t box_rows(bool fp8, int gemm) {
 template <bool FP8, bool NARROW>
 cudaError_t set_pair_attrs() {
   using P = GemmPair<FP8, NARROW>;
-  cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false>();
-  if (e != cudaSuccess) return e;
-  return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split>();
+  if constexpr (P::fused) {
+    return set_gemm_attr<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>();
+  } else {
+    cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false>();
+    if (e != cudaSuccess) return e;
+    return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split>();
+  }
 }
 
 template <bool FP8>
@@ -265,8 +290,10 @@ cudaError_t set_all_gemm_attrs() {
 }
 
 template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
-void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
-  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, 192, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, args);
+void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
+                 const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
+  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, 192, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
+      a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
 }
 
 // K split of the tensor-core router: enough units to cover the SMs, every split non-empty.
@@ -360,6 +387,26 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g1.a_scale = h->w.w13_scale;
   g1.b_scale = h->xscale;
   g1.err = h->err;
+  if constexpr (P::fused) {
+    // one launch: gate/up units then down units, down units gated by the act-tile counters
+    GemmArgs f = g1;
+    f.unit_base2 = h->ub2;
+    f.tile_base = h->tile_base;
+    f.tile_done = h->tile_done;
+    f.K2 = c.I;
+    f.a_rows2 = c.H;
+    f.mt_stride2 = 256;
+    f.second_off2 = 128;
+    f.out2 = h->Y;
+    f.out_ld2 = c.H;
+    f.mt1 = c.I / 128;
+    record(h, 5, s);
+    launch_gemm<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>(h->num_sms, h->tm_w13, h->tm_xp[shape], f, s,
+                                                                &h->tm_w2, &h->tm_act[shape]);
+    record(h, 6, s);
+    record(h, 7, s);
+    return;
+  }
   record(h, 5, s);
   launch_gemm<P::bn1, P::st1, FP8, 0, false>(h->num_sms, h->tm_w13, h->tm_xp[shape], g1, s);
   record(h, 6, s);
@@ -392,7 +439,8 @@ int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream
   }
   record(h, 4, s);
   build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn1, bn2, c.I / 128, c.H / 256,
-                                          h->grp_rows, h->grp_base, h->ub1, h->ub2, h->err);
+                                          h->grp_rows, h->grp_base, h->ub1, h->ub2, h->tile_base, h->tile_done,
+                                          h->err);
   if (h->fp8) {
     if (narrow) run_gemms<true, true>(h, T, s);
     else run_gemms<true, false>(h, T, s);
@@ -525,6 +573,8 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
       {reinterpret_cast<void**>(&h->grp_base), static_cast<size_t>(h->G) * 4},
       {reinterpret_cast<void**>(&h->ub1), static_cast<size_t>(h->G + 1) * 4},
       {reinterpret_cast<void**>(&h->ub2), static_cast<size_t>(h->G + 1) * 4},
+      {reinterpret_cast<void**>(&h->tile_base), static_cast<size_t>(h->G) * 4},
+      {reinterpret_cast<void**>(&h->tile_done), static_cast<size_t>(R / 16 + h->G + 1) * 4},
       {reinterpret_cast<void**>(&h->xp), R * c.H * wb},
       {reinterpret_cast<void**>(&h->xscale), R * 4},
       {&act_p, R * c.I * 4},  // fp32 (W8A8) or two bf16 planes (hi, lo)

@@ -232,11 +232,14 @@ quantize_act_kernel(const float* __restrict__ act32, int R, int I, uint8_t* __re
 // group E is the shared expert (rows T*k .. T*k + T).  Each group contributes
 // ceil(rows / bn1) * mt1 tile units to the gate/up GEMM and ceil(rows / bn2) * mt2 to the
 // down GEMM; unit bases are exclusive prefix sums.  One CTA of 512 threads (G <= 257).
+// Also: tile_base[g] = first N tile (of bn1 rows) of group g, and the per-tile counters of the
+// fused kernel's act dependencies are zeroed.
 __global__ void __launch_bounds__(512)
 build_schedule_kernel(const int32_t* __restrict__ offsets, int E, int n_shared, int T, int k, int bn1, int bn2,
                       int mt1, int mt2, int32_t* __restrict__ grp_rows, int32_t* __restrict__ grp_base,
-                      int32_t* __restrict__ ub1, int32_t* __restrict__ ub2, int* err) {
-  __shared__ int wsum1[16], wsum2[16];
+                      int32_t* __restrict__ ub1, int32_t* __restrict__ ub2, int32_t* __restrict__ tile_base,
+                      int* __restrict__ tile_done, int* err) {
+  __shared__ int wsum1[16], wsum2[16], wsum3[16];
   const int g = threadIdx.x, lane = g & 31, warp = g >> 5;
   const int G = E + n_shared;
   int rows = 0, rbase = 0;
@@ -252,22 +255,25 @@ build_schedule_kernel(const int32_t* __restrict__ offsets, int E, int n_shared, 
     rows = T;
     rbase = T * k;  // shared-expert rows follow the routed rows
   }
-  const int u1 = (rows + bn1 - 1) / bn1 * mt1, u2 = (rows + bn2 - 1) / bn2 * mt2;
-  const int i1 = warp_incl_scan(u1, lane), i2 = warp_incl_scan(u2, lane);
-  if (lane == 31) { wsum1[warp] = i1; wsum2[warp] = i2; }
+  const int nt = (rows + bn1 - 1) / bn1;
+  const int u1 = nt * mt1, u2 = (rows + bn2 - 1) / bn2 * mt2;
+  const int i1 = warp_incl_scan(u1, lane), i2 = warp_incl_scan(u2, lane), i3 = warp_incl_scan(nt, lane);
+  if (lane == 31) { wsum1[warp] = i1; wsum2[warp] = i2; wsum3[warp] = i3; }
   __syncthreads();
   if (warp == 0) {
-    const int a = lane < 16 ? wsum1[lane] : 0, b = lane < 16 ? wsum2[lane] : 0;
-    const int ia = warp_incl_scan(a, lane), ib = warp_incl_scan(b, lane);
-    if (lane < 16) { wsum1[lane] = ia - a; wsum2[lane] = ib - b; }
+    const int a = lane < 16 ? wsum1[lane] : 0, b = lane < 16 ? wsum2[lane] : 0, c = lane < 16 ? wsum3[lane] : 0;
+    const int ia = warp_incl_scan(a, lane), ib = warp_incl_scan(b, lane), ic = warp_incl_scan(c, lane);
+    if (lane < 16) { wsum1[lane] = ia - a; wsum2[lane] = ib - b; wsum3[lane] = ic - c; }
   }
   __syncthreads();
-  const int e1 = wsum1[warp] + i1 - u1, e2 = wsum2[warp] + i2 - u2;
+  const int e1 = wsum1[warp] + i1 - u1, e2 = wsum2[warp] + i2 - u2, e3 = wsum3[warp] + i3 - nt;
   if (g < G) {
     grp_rows[g] = rows;
     grp_base[g] = rbase;
     ub1[g] = e1;
     ub2[g] = e2;
+    tile_base[g] = e3;
+    for (int i = 0; i < nt; ++i) tile_done[e3 + i] = 0;
   }
   if (g == G - 1) {
     ub1[G] = e1 + u1;

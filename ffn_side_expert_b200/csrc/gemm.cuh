@@ -20,6 +20,13 @@
 // split of Henry, Tang and Heinecke, "Leveraging the bfloat16 AI datatype for higher-precision
 // computations", 2019).  The only bf16 rounding left on the output path is the layer output.
 //
+// MODE 3 (fused, bf16): gate/up units and down units in ONE persistent launch.  Every CTA takes
+// its gate/up units first, then its down units.  A gate/up epilogue publishes each finished act
+// tile with a release increment of its (expert, N tile) counter; the producer of a down unit
+// waits (acquire, bounded) until all I/128 act tiles of its rows are in, then issues its loads.
+// Every dependency lies earlier in each CTA's unit order, so the waits always end; the HBM-bound
+// weight stream of late gate/up units overlaps the tensor-heavier down units.
+//
 // MODE 2 (router): the fp32 router weights are stored once as three bf16 planes hi + mid + lo
 // (each the bf16 rounding of what the previous planes leave), so Wr is represented to ~2^-27
 // relative; bf16 x bf16 products are exact in fp32 and the three planes accumulate into one
@@ -69,10 +76,18 @@ struct GemmArgs {
   const float* a_scale;      // W8A8: per weight row [G * a_rows]
   const float* b_scale;      // W8A8: per token row [R]
   int* err;                  // device error word
+  // MODE 3 (fused): the down GEMM's side and the act-tile dependency counters
+  const int32_t* unit_base2; // [G+1] units of the down GEMM
+  const int32_t* tile_base;  // [G] first N tile of each group
+  int* tile_done;            // [N tiles] gate/up units finished per (group, N tile)
+  int K2, a_rows2, mt_stride2, second_off2, out_ld2;
+  void* out2;                // Y
+  int mt1;                   // gate/up units per N tile (I / 128)
 };
 
 template <int BN, bool SPLIT_B = false, int MODE = 0>
 struct GemmShape {
+  static constexpr bool kFused = MODE == 3;
   static constexpr int kNA = MODE == 2 ? 3 : 2;         // weight tiles per stage
   static constexpr int kNDU = MODE == 2 ? 1 : 2;        // accumulators per unit
   static constexpr int kATile = 128 * 128;              // one 128-row x 128-byte weight tile
@@ -87,8 +102,10 @@ struct GemmShape {
   static constexpr bool kConcat = SPLIT_B && BN <= AFD_CONCAT_MAX_BN;
   // rows per TMA box of a token tile: few large boxes keep the single producer thread from
   // becoming the bottleneck; a box may overrun the unit's rows (the MMA reads only n16 rows)
-  // except in the concatenated layout, where the lo rows follow the hi rows directly
-  static constexpr int kBoxRows = kConcat ? (BN <= 32 ? 16 : 32) : (BN < 64 ? BN : 64);
+  // except in the concatenated layout, where the lo rows follow the hi rows directly.
+  // kBoxRowsX: single-plane token tiles (the gate/up side of the fused kernel)
+  static constexpr int kBoxRowsX = BN < 64 ? BN : 64;
+  static constexpr int kBoxRows = kConcat ? (BN <= 32 ? 16 : 32) : kBoxRowsX;
   // concatenated layout: hi rows padded to whole boxes, then the lo rows
   __device__ static int npad(int n16) { return kConcat ? (n16 + kBoxRows - 1) / kBoxRows * kBoxRows : n16; }
   static constexpr int kUnitCols = kNDU * BN * (kConcat ? 2 : 1);  // TMEM columns of one unit
@@ -108,8 +125,8 @@ constexpr int kSchedBytes = (kMaxGroups + 1) * 16;
 
 template <int BN, int STAGES, bool SPLIT_B, int MODE = 0>
 constexpr int gemm_smem_bytes() {
-  return kSchedBytes + 1024 /*alignment slack*/ + STAGES * GemmShape<BN, SPLIT_B, MODE>::kStageBytes +
-         256 /*barriers*/;
+  return (MODE == 3 ? 2 : 1) * kSchedBytes + 1024 /*alignment slack*/ +
+         STAGES * GemmShape<BN, SPLIT_B, MODE>::kStageBytes + 256 /*barriers*/;
 }
 
 // Largest g with tab[g].x (first unit of group g) <= u; the table sits in shared memory.
@@ -125,11 +142,23 @@ __device__ __forceinline__ int find_group(const int4* tab, int G, int u) {
 struct Unit {
   int g, mt, rows, row0, n16;  // group, tile pair, valid token rows, first row, MMA N
   int kc0, kc1, split;         // K chunks [kc0, kc1) and their split index
+  int mode, tile;              // 0 gate/up, 1 down, 2 router; (group, N tile) id for MODE 3
 };
 
-template <int BN>
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, int u, int kchunks) {
+template <int BN, int MODE>
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, const int4* tab2, int u,
+                                           int kchunks, int kchunks2) {
   Unit w;
+  w.mode = MODE == 3 ? 0 : MODE;
+  if constexpr (MODE == 3) {
+    const int u1 = tab[a.G].x;
+    if (u >= u1) {  // a down unit
+      u -= u1;
+      tab = tab2;
+      kchunks = kchunks2;
+      w.mode = 1;
+    }
+  }
   if (a.single_rows >= 0) {
     const int ntiles = (a.single_rows + BN - 1) / BN;
     const int per_split = ntiles * a.single_mt;
@@ -142,6 +171,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, 
     w.row0 = nt * BN;
     w.kc0 = w.split * a.kc_per;
     w.kc1 = min(kchunks, w.kc0 + a.kc_per);
+    w.tile = 0;
   } else {
     w.g = find_group(tab, a.G, u);
     const int4 gs = tab[w.g];
@@ -155,6 +185,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, 
     w.split = 0;
     w.kc0 = 0;
     w.kc1 = kchunks;
+    w.tile = gs.w + nt;
   }
   w.n16 = (w.rows + 15) & ~15;
   return w;
@@ -162,27 +193,51 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, 
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until the gate/up units of a down unit's rows are all published (bounded like mbar_wait),
+// then order the async-proxy (TMA) reads that follow after them.
+__device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int* abort) {
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(cnt) < need) {
+    if (*abort || clock64() - t0 > kWaitLimitCycles) return false;
+    __nanosleep(64);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B>
 __global__ void __launch_bounds__(192, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs args) {
-  static_assert(!(SPLIT_B && (FP8 || MODE != 1)), "two-term B only for the bf16 down GEMM");
-  static_assert(!(MODE == 2 && FP8), "the router runs on bf16 planes");
+  static_assert(!(SPLIT_B && (FP8 || (MODE != 1 && MODE != 3))), "two-term B only for the bf16 down GEMM");
+  static_assert(!((MODE == 2 || MODE == 3) && FP8), "router and fused modes run on bf16");
   using S = GemmShape<BN, SPLIT_B, MODE>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
 
   extern __shared__ uint8_t smem_raw[];
   int4* sched = reinterpret_cast<int4*>(smem_raw);  // group schedule copy
-  const uint32_t raw = smem_u32(smem_raw) + kSchedBytes;
+  int4* sched2 = sched + (kMaxGroups + 1);          // MODE 3: the down GEMM's schedule
+  constexpr int kSchedAll = (MODE == 3 ? 2 : 1) * kSchedBytes;
+  const uint32_t raw = smem_u32(smem_raw) + kSchedAll;
   const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + kSchedBytes + (base - raw);
+  uint8_t* gbase = smem_raw + kSchedAll + (base - raw);
   const uint32_t bars = base + STAGES * S::kStageBytes;
   // barrier block: full[STAGES], empty[STAGES], tfull[kNacc], tempty[kNacc], done
   const uint32_t full = bars, empty = bars + 8u * STAGES;
   const uint32_t tfull = bars + 16u * STAGES, tempty = tfull + 8u * kNacc;
   const uint32_t done_bar = tempty + 8u * kNacc;
-  constexpr int kBars = 2 * STAGES + 2 * kNacc + 1;
+  // MODE 3: per accumulator buffer, the four epilogue warps finished an act tile.  A warp arrives
+  // here before it releases the buffer, so the next unit on the same buffer cannot arrive early.
+  const uint32_t epi_bar = done_bar + 8u;
+  constexpr int kBars = 2 * STAGES + 3 * kNacc + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStageBytes + 8 * kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -199,27 +254,40 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_init(tempty + 8u * i, 4);
     }
     mbar_init(done_bar, 1);
+    for (int i = 0; i < kNacc; ++i) mbar_init(epi_bar + 8u * i, 4);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if constexpr (MODE == 3) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
     tmem_relinquish();
   }
   if (args.single_rows < 0) {
-    for (int g = threadIdx.x; g <= args.G; g += blockDim.x)
-      sched[g] = g < args.G ? make_int4(__ldg(args.unit_base + g), __ldg(args.grp_rows + g), __ldg(args.grp_base + g), 0)
+    for (int g = threadIdx.x; g <= args.G; g += blockDim.x) {
+      const int tb = (MODE == 3 && g < args.G) ? __ldg(args.tile_base + g) : 0;
+      sched[g] = g < args.G ? make_int4(__ldg(args.unit_base + g), __ldg(args.grp_rows + g), __ldg(args.grp_base + g), tb)
                             : make_int4(__ldg(args.unit_base + g), 0, 0, 0);
+      if constexpr (MODE == 3)
+        sched2[g] = g < args.G ? make_int4(__ldg(args.unit_base2 + g), __ldg(args.grp_rows + g),
+                                           __ldg(args.grp_base + g), tb)
+                               : make_int4(__ldg(args.unit_base2 + g), 0, 0, 0);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int total = args.single_rows >= 0 ? args.single_total : sched[args.G].x;
+  const int total = args.single_rows >= 0 ? args.single_total
+                                          : sched[args.G].x + (MODE == 3 ? sched2[args.G].x : 0);
   const int kchunks = args.K / kKChunk;
+  const int kchunks2 = MODE == 3 ? args.K2 / kKChunk : kchunks;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -228,13 +296,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     int issued = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit w = decode_unit<BN>(args, sched, u, kchunks);
-      const int ya = w.g * args.a_rows + w.mt * args.mt_stride;
-      const int nbox = (w.n16 + S::kBoxRows - 1) / S::kBoxRows;  // token-tile boxes per plane
-      const uint32_t tx = S::kAStage + (SPLIT_B ? 2u : 1u) * static_cast<uint32_t>(nbox * S::kBoxRows) * 128u;
+      const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
+      // the down side of the fused kernel uses the second set of maps and coordinates
+      const bool down = MODE == 3 && w.mode == 1;
+      const CUtensorMap* mA = down ? &tmA2 : &tmA;
+      const CUtensorMap* mB = down ? &tmB2 : &tmB;
+      const int ya = down ? w.g * args.a_rows2 + w.mt * args.mt_stride2 : w.g * args.a_rows + w.mt * args.mt_stride;
+      const int soff = down ? args.second_off2 : args.second_off;
+      const bool two = SPLIT_B && (MODE != 3 || down);           // hi and lo planes
+      const int boxr = (MODE == 3 && !down) ? S::kBoxRowsX : S::kBoxRows;
+      const int nbox = (w.n16 + boxr - 1) / boxr;                  // token-tile boxes per plane
+      const uint32_t tx = S::kAStage + (two ? 2u : 1u) * static_cast<uint32_t>(nbox * boxr) * 128u;
       // the lo activation rows follow the (padded) hi rows or sit one tile further
       const uint32_t lo_off = S::kConcat ? static_cast<uint32_t>(S::npad(w.n16)) * 128u : S::kBTile;
       const uint64_t apol = MODE == 2 ? kEvictLast : args.a_policy;
+      if (down && !wait_tile(args.tile_done + w.tile, args.mt1, abort_flag)) { ok = false; break; }
       for (int kc = w.kc0; kc < w.kc1; ++kc) {
         if (!mbar_wait(empty + 8u * s, ph ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t st = base + s * S::kStageBytes;
@@ -244,14 +320,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // the pair (MODE 0/1) or the three router planes (MODE 2), second_off apart
 #pragma unroll
         for (int i = 0; i < S::kNA; ++i)
-          tma_load_2d(st + i * S::kATile, &tmA, fb, x, ya + i * args.second_off, apol);
+          tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
         const uint32_t sb = st + S::kAStage;
         for (int b = 0; b < nbox; ++b)
-          tma_load_2d(sb + b * S::kBoxRows * 128, &tmB, fb, x, w.row0 + b * S::kBoxRows, kEvictLast);
-        if constexpr (SPLIT_B) {
+          tma_load_2d(sb + b * boxr * 128, mB, fb, x, w.row0 + b * boxr, kEvictLast);
+        if (two) {
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sb + lo_off + b * S::kBoxRows * 128, &tmB, fb, x, args.lo_rows + w.row0 + b * S::kBoxRows,
-                        kEvictLast);
+            tma_load_2d(sb + lo_off + b * boxr * 128, mB, fb, x, args.lo_rows + w.row0 + b * boxr, kEvictLast);
         }
         ++issued;
         if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -272,8 +347,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t acc_ph = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit w = decode_unit<BN>(args, sched, u, kchunks);
-      const uint32_t idesc = idesc_m128(S::kConcat ? 2 * S::npad(w.n16) : w.n16, FP8);
+      const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
+      const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
+      const bool cat = S::kConcat && down;
+      const uint32_t idesc = idesc_m128(cat ? 2 * S::npad(w.n16) : w.n16, FP8);
       if (!mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d0 = tmem + static_cast<uint32_t>(acc * S::kUnitCols);
@@ -297,9 +374,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_mma<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
             if constexpr (SPLIT_B && !S::kConcat) {  // the lo plane as separate MMAs
-              const uint64_t dl = sw128_desc(st + S::kAStage + S::kBTile);
-              tc_mma<FP8>(d0, da0 + 2 * kk, dl + 2 * kk, idesc, 1u);
-              tc_mma<FP8>(d1, da1 + 2 * kk, dl + 2 * kk, idesc, 1u);
+              if (down) {
+                const uint64_t dl = sw128_desc(st + S::kAStage + S::kBTile);
+                tc_mma<FP8>(d0, da0 + 2 * kk, dl + 2 * kk, idesc, 1u);
+                tc_mma<FP8>(d1, da1 + 2 * kk, dl + 2 * kk, idesc, 1u);
+              }
             }
           }
         }
@@ -321,8 +400,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int m = q * 32 + lane;          // row within the 128-row weight tile
     int acc = 0;
     uint32_t acc_ph = 0;
+    uint32_t epi_ph = 0;  // parity bit per accumulator buffer
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit w = decode_unit<BN>(args, sched, u, kchunks);
+      const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       if (!mbar_wait(tfull + 8u * acc, acc_ph, abort_flag)) {
         *abort_flag = 1;
         atomicOr(args.err, kErrTimeout);
@@ -332,8 +412,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t t0 = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::kUnitCols);
       const uint32_t t1 = t0 + S::kUnitCols / 2;
       // weight rows of this thread in the two tiles
-      const int wrow0 = w.mt * args.mt_stride + m;
-      const int wrow1 = wrow0 + args.second_off;
+      const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
+      const int wrow0 = w.mt * (MODE == 3 && down ? args.mt_stride2 : args.mt_stride) + m;
+      const int wrow1 = wrow0 + (MODE == 3 && down ? args.second_off2 : args.second_off);
       if constexpr (MODE == 2) {  // partial logits [split][t][e]; rows past E are padding
         const int e = wrow0;
         float* lg = static_cast<float*>(args.out) + static_cast<size_t>(w.split) * args.single_rows * args.out_ld;
@@ -359,7 +440,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tmem_ld16(t0 + c, r0);
           tmem_ld16(t1 + c, r1);
           tmem_ld_wait(r0, r1);
-          if constexpr (S::kConcat) {  // add the lo-plane half (columns npad..) of each tile
+          if (S::kConcat && down) {  // add the lo-plane half (columns npad..) of each tile
             uint32_t l0[16], l1[16];
             tmem_ld16(t0 + S::npad(w.n16) + c, l0);
             tmem_ld16(t1 + S::npad(w.n16) + c, l1);
@@ -382,7 +463,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 v0 = v0 * sa0 * sb;
                 v1 = v1 * sa1 * sb;
               }
-              if constexpr (MODE == 0) {
+              if (!down) {
                 const float act = silu_f(v0) * v1;  // gate tile first, up tile second
                 if constexpr (FP8) {
                   static_cast<float*>(args.out)[row * args.out_ld + wrow0] = act;
@@ -398,7 +479,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 y[wrow0] = __float2bfloat16_rn(v0);
                 y[wrow1] = __float2bfloat16_rn(v1);
               } else {
-                float* y = static_cast<float*>(args.out) + row * args.out_ld;
+                float* y = static_cast<float*>(MODE == 3 ? args.out2 : args.out) +
+                           row * (MODE == 3 ? args.out_ld2 : args.out_ld);
                 y[wrow0] = v0;
                 y[wrow1] = v1;
               }
@@ -408,6 +490,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       tc_fence_before();
       __syncwarp();
+      if constexpr (MODE == 3) {
+        if (!down) {  // publish this act tile once all four epilogue warps have stored their rows
+          const uint32_t eb = epi_bar + 8u * acc;
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // stores above -> later TMA reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(eb);
+          if (warp == 2 && lane == 0) {
+            if (mbar_wait(eb, (epi_ph >> acc) & 1u, abort_flag)) {
+              __threadfence();
+              atomicAdd(args.tile_done + w.tile, 1);
+            } else {
+              *abort_flag = 1;
+              atomicOr(args.err, kErrTimeout);
+            }
+          }
+          epi_ph ^= 1u << acc;
+        }
+      }
       if (lane == 0) mbar_arrive(tempty + 8u * acc);
       if (++acc == kNacc) { acc = 0; acc_ph ^= 1u; }
     }
