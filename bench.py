@@ -34,14 +34,15 @@ import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the gate/up GEMM with the
-# decode tile shape, from the ncu capture in profiles/grouped_gemm_decode_T16_E16.md
-# (1 003 994 112 B for 272 weight-tile pairs: 17 expert groups x 16).  Traffic grows with the
-# distinct weight tiles streamed (the N tiles of one weight tile share it through L2), and it is
-# reported only while gemm.cuh is the source that was captured.
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
+# of the decode shape, from a one-pass ncu capture of two launches at T=256, H=7168, E=256,
+# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 068 632 320 and
+# 23 060 022 272 bytes for 257 touched experts.  Traffic grows with the experts whose weights
+# are streamed, and it is reported only while the kernel source and its instantiation are the
+# ones that were captured.
 MEASURED_TRAFFIC = {
-    "gemm_cuh_sha256": "6c6cb4e38901f8072a1cf0c878daf423345437ea7548b923ab12f5b5630f4a24",
-    "bytes_per_unit": 1003994112 / 272,
+    "sources_sha256": "3b01a3473e3a27d2e5c30d7711436fc452ca3def330c9ffc2a194d9ac53678cf",
+    "bytes_per_touched_expert": (23068632320 + 23060022272) / 2 / 257,
 }
 METRIC = "MoE-FFN tokens/s/layer"
 
@@ -70,24 +71,26 @@ def algorithmic(cfg, counts) -> dict:
     # the fused bf16 expert kernel (gate/up + SwiGLU + down): weights, dispatched rows in, outputs out
     expert = w13 + w2 + rows * H * b + rows * H * 4
     flops = 6 * H * I * (T * k + S * T) + 2 * T * H * E
-    units = n * (I // 128)   # distinct gate/up weight-tile pairs streamed
     return {"weight_bytes": w13 + w2, "act_bytes": act, "flops": flops, "gemm13_bytes": gemm13,
             "expert_bytes": expert,
-            "gemm13_flops": 4 * H * I * rows, "touched_experts": n, "gemm13_units_narrow": units}
+            "gemm13_flops": 4 * H * I * rows, "touched_experts": n}
 
 
-def gate_up_traffic(cfg, acct):
-    """Measured DRAM bytes per gate/up launch scaled to this workload, or None when the kernel
-    source changed since the capture or the launch uses another tile shape or dtype."""
+def kernel_sources_sha256() -> str:
     import hashlib
-    path = os.path.join(ROOT, "ffn_side_expert_b200", "csrc", "gemm.cuh")
-    with open(path, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    narrow = cfg.T * cfg.k <= 32 * cfg.E
-    if sha != MEASURED_TRAFFIC["gemm_cuh_sha256"] or cfg.dtype != "bf16" or not narrow:
+    h = hashlib.sha256()
+    for name in ("gemm.cuh", "afd_ffn.cu"):
+        with open(os.path.join(ROOT, "ffn_side_expert_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def fused_traffic(cfg, acct):
+    """Measured DRAM bytes per fused expert-kernel launch scaled to this workload's touched
+    experts, or None when the kernel sources changed since the capture."""
+    if kernel_sources_sha256() != MEASURED_TRAFFIC["sources_sha256"]:
         return None
-    units = acct["gemm13_units_narrow"]
-    return int(round(MEASURED_TRAFFIC["bytes_per_unit"] * units))
+    return int(round(MEASURED_TRAFFIC["bytes_per_touched_expert"] * acct["touched_experts"]))
 
 
 def load_peaks():
@@ -311,11 +314,11 @@ def report_ours(args, world, r) -> dict:
     if cfg.dtype == "bf16" and cfg.T * cfg.k <= 32 * cfg.E:  # decode shape: one fused launch
         kname, kbytes = "expert FFN kernel (gate/up + SwiGLU + down, fused)", acct["expert_bytes"]
         k_ms = stage["gemm_gate_up"] + stage["gemm_down"]
-        traffic = None
+        traffic = fused_traffic(cfg, acct)
     else:
         kname, kbytes = "grouped_gemm gate/up + SwiGLU", acct["gemm13_bytes"]
         k_ms = stage["gemm_gate_up"]
-        traffic = gate_up_traffic(cfg, acct)
+        traffic = None
     achieved = kbytes / (k_ms / 1e3) / 1e9
     t_hbm = (acct["weight_bytes"] + acct["act_bytes"]) / (hbm * 1e9)
     tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.dtype == "fp8" else 1.0)

@@ -292,7 +292,7 @@ cudaError_t set_all_gemm_attrs() {
 template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
 void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
                  const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
-  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, 192, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
+  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
       a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
 }
 

@@ -34,9 +34,12 @@
 // in order by the top-k kernel) to spread a small micro-batch over more SMs.
 //
 // Pipeline: one ring of STAGES shared-memory stages, each holding the weight tiles and the
-// token tile of one 128-byte K chunk.  Warp roles (192 threads): warp 0 lane 0 issues the TMA
-// loads, warp 1 owns the TMEM allocation and its lane 0 issues tcgen05.mma (one commit per
-// stage), warps 2..5 are the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// token tile of one 128-byte K chunk.  Warp roles (64 + 32 x kEpiWarps threads): warp 0 lane 0
+// issues the TMA loads, warp 1 owns the TMEM allocation and its lane 0 issues tcgen05.mma (one
+// commit per stage), warps 2.. are the epilogue.  An epilogue warp w reads TMEM lanes
+// 32*(w%4)..+31 (the lane quarter the hardware lets it access); with 8 epilogue warps two warps
+// share each quarter and take alternate 16-column chunks, so every scheduler runs two epilogue
+// warps and the SwiGLU / scaling math of one unit overlaps the next unit's MMAs.
 // Decode shape of the bf16 down GEMM: the hi and lo activation rows of a stage sit back to
 // back, so one MMA of N = 2 x rows covers both planes and the epilogue adds the two halves --
 // half the MMA instructions of issuing each plane separately, which matters when every MMA is
@@ -191,7 +194,16 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, 
   return w;
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+// silu(z) = z / (1 + e^-z) with the fast exponential and division intrinsics (relative error of
+// a few 1e-7 over the range that matters; the limit z -> -inf gives -0).
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+#ifndef AFD_EPI_WARPS
+#define AFD_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = AFD_EPI_WARPS;          // 4 or 8
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -212,7 +224,7 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
 }
 
 template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs args) {
@@ -251,10 +263,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int i = 0; i < kNacc; ++i) {
       mbar_init(tfull + 8u * i, 1);
-      mbar_init(tempty + 8u * i, 4);
+      mbar_init(tempty + 8u * i, kEpiWarps);
     }
     mbar_init(done_bar, 1);
-    for (int i = 0; i < kNacc; ++i) mbar_init(epi_bar + 8u * i, 4);
+    for (int i = 0; i < kNacc; ++i) mbar_init(epi_bar + 8u * i, kEpiWarps);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -394,10 +406,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tc_commit(done_bar);
     volatile int never = 0;
     mbar_wait(done_bar, 0, &never);
-  } else if (warp >= 2 && warp <= 5) {
+  } else if (warp >= 2 && warp < 2 + kEpiWarps) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;               // TMEM lane quarter of this warp
     const int m = q * 32 + lane;          // row within the 128-row weight tile
+    constexpr int kCStep = 16 * (kEpiWarps / 4);  // the column chunks of the warps sharing q
+    const int c_first = 16 * ((warp - 2) / 4);
     int acc = 0;
     uint32_t acc_ph = 0;
     uint32_t epi_ph = 0;  // parity bit per accumulator buffer
@@ -418,7 +432,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if constexpr (MODE == 2) {  // partial logits [split][t][e]; rows past E are padding
         const int e = wrow0;
         float* lg = static_cast<float*>(args.out) + static_cast<size_t>(w.split) * args.single_rows * args.out_ld;
-        for (int c = 0; c < w.n16; c += 16) {
+        for (int c = c_first; c < w.n16; c += kCStep) {
           uint32_t r0[16];
           tmem_ld16(t0 + c, r0);
           tmem_ld_wait(r0);
@@ -435,7 +449,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           sa0 = __ldg(args.a_scale + static_cast<size_t>(w.g) * args.a_rows + wrow0);
           sa1 = __ldg(args.a_scale + static_cast<size_t>(w.g) * args.a_rows + wrow1);
         }
-        for (int c = 0; c < w.n16; c += 16) {
+        for (int c = c_first; c < w.n16; c += kCStep) {
+          // W8A8: lane i < 16 fetches the scale of token c + i once; shuffled to all lanes below
+          float sb_lane = 0.f;
+          if constexpr (FP8) {
+            if (lane < 16 && c + lane < w.rows) sb_lane = __ldg(args.b_scale + w.row0 + c + lane);
+          }
           uint32_t r0[16], r1[16];
           tmem_ld16(t0 + c, r0);
           tmem_ld16(t1 + c, r1);
@@ -454,12 +473,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int n = c + i;
+            float sb = 1.f;
+            if constexpr (FP8) sb = __shfl_sync(0xffffffffu, sb_lane, i);
             if (n < w.rows) {
               const size_t row = static_cast<size_t>(w.row0 + n);
               float v0 = __uint_as_float(r0[i]);
               float v1 = __uint_as_float(r1[i]);
               if constexpr (FP8) {
-                const float sb = __ldg(args.b_scale + row);
                 v0 = v0 * sa0 * sb;
                 v1 = v1 * sa1 * sb;
               }
