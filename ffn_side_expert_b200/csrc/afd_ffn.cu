@@ -42,6 +42,7 @@ struct afd_ffn_handle {
   afd_ffn_weights w;
   int device = 0;
   int num_sms = 0;
+  int pair_grid = 0;  // CTAs of the CTA-pair GEMMs: 2 x the pairs that fit on the device at once
   bool fp8 = false;
   int G = 0;       // E + n_shared
   int R_max = 0;   // rows of the dispatched-row buffers: T_max * (k + 1)
@@ -158,10 +159,11 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, ST, SPLIT, MODE>());
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gemm_smem_bytes<BN, ST, SPLIT, MODE, PAIR>());
 }
 
 // (gate/up, down) kernel pairs of each path and tile shape: N tile and ring stages of each
@@ -180,19 +182,26 @@ cudaError_t set_gemm_attr() {
 #ifndef AFD_NB_G2_ST
 #define AFD_NB_G2_ST 5
 #endif
+// AFD_WIDE_PAIR=1 runs each large-micro-batch unit on a CTA pair (2-CTA cluster, M = 256 pair
+// MMAs, N = BN token rows split between the two CTAs): per CTA a 48 KB stage then feeds twice
+// the MMA work of a one-CTA 128 x 128 unit.  Measured on B200 it is slower than one CTA per unit
+// (W8A8 T=8192: 5.04 vs 4.72 ms; bf16 T=4096: 6.03 vs 5.78 ms), so it is off by default.
+#ifndef AFD_WIDE_PAIR
+#define AFD_WIDE_PAIR 0
+#endif
 // bf16 large micro-batch, gate/up
 #ifndef AFD_WB_G1_BN
-#define AFD_WB_G1_BN 128
+#define AFD_WB_G1_BN (AFD_WIDE_PAIR ? 256 : 128)
 #endif
 #ifndef AFD_WB_G1_ST
 #define AFD_WB_G1_ST 4
 #endif
 // bf16 large micro-batch, down (two activation planes per stage)
 #ifndef AFD_WB_G2_BN
-#define AFD_WB_G2_BN 128
+#define AFD_WB_G2_BN (AFD_WIDE_PAIR ? 256 : 128)
 #endif
 #ifndef AFD_WB_G2_ST
-#define AFD_WB_G2_ST 3
+#define AFD_WB_G2_ST (AFD_WIDE_PAIR ? 4 : 3)
 #endif
 // W8A8 decode, gate/up
 #ifndef AFD_NF_G1_BN
@@ -210,17 +219,17 @@ cudaError_t set_gemm_attr() {
 #endif
 // W8A8 large micro-batch, gate/up
 #ifndef AFD_WF_G1_BN
-#define AFD_WF_G1_BN 128
+#define AFD_WF_G1_BN (AFD_WIDE_PAIR ? 256 : 128)
 #endif
 #ifndef AFD_WF_G1_ST
 #define AFD_WF_G1_ST 4
 #endif
 // W8A8 large micro-batch, down
 #ifndef AFD_WF_G2_BN
-#define AFD_WF_G2_BN 128
+#define AFD_WF_G2_BN (AFD_WIDE_PAIR ? 256 : 128)
 #endif
 #ifndef AFD_WF_G2_ST
-#define AFD_WF_G2_ST 4
+#define AFD_WF_G2_ST (AFD_WIDE_PAIR ? 6 : 4)
 #endif
 
 // bf16 decode shape: the gate/up and down GEMMs run fused in one launch (MODE 3) with stf ring
@@ -237,63 +246,142 @@ cudaError_t set_gemm_attr() {
 #define AFD_WB_F_ST 0
 #endif
 
-template <int BN1, int ST1, int BN2, int ST2, bool SPLIT, int STF = 0>
+template <int BN1, int ST1, int BN2, int ST2, bool SPLIT, int STF = 0, bool PAIR = false>
 struct GemmPairT {
   static constexpr int bn1 = BN1, st1 = ST1, bn2 = BN2, st2 = ST2;
   static constexpr int stf = STF;
   static constexpr bool split = SPLIT;
-  static constexpr bool fused = STF > 0 && BN1 == BN2 && AFD_FUSED;
+  static constexpr bool pair = PAIR;  // both GEMMs on CTA pairs
+  static constexpr bool fused = !PAIR && STF > 0 && BN1 == BN2 && AFD_FUSED;
+  // gate/up units per N tile: 128 gate rows (+ up) per unit, or 256 on a pair
+  static constexpr int gate_rows_per_unit = PAIR ? 256 : 128;
 };
-template <bool FP8, bool NARROW>
+// Tile shapes: kNarrow (decode), kWide (large micro-batch on CTA pairs when I % 256 == 0) and
+// kWideSingle (large micro-batch, one CTA per unit: any I that is a multiple of 128).
+constexpr int kNarrow = 0, kWide = 1, kWideSingle = 2;
+template <bool FP8, int SHAPE>
 struct GemmPair;
 template <>
-struct GemmPair<false, true>
+struct GemmPair<false, kNarrow>
     : GemmPairT<AFD_NB_G1_BN, AFD_NB_G1_ST, AFD_NB_G2_BN, AFD_NB_G2_ST, true, AFD_NB_F_ST> {};
 template <>
-struct GemmPair<false, false>
-    : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true, AFD_WB_F_ST> {};
+struct GemmPair<false, kWide>
+    : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true, AFD_WB_F_ST, AFD_WIDE_PAIR> {};
 template <>
-struct GemmPair<true, true> : GemmPairT<AFD_NF_G1_BN, AFD_NF_G1_ST, AFD_NF_G2_BN, AFD_NF_G2_ST, false> {};
+struct GemmPair<false, kWideSingle> : GemmPairT<128, 4, 128, 3, true> {};
 template <>
-struct GemmPair<true, false> : GemmPairT<AFD_WF_G1_BN, AFD_WF_G1_ST, AFD_WF_G2_BN, AFD_WF_G2_ST, false> {};
+struct GemmPair<true, kNarrow> : GemmPairT<AFD_NF_G1_BN, AFD_NF_G1_ST, AFD_NF_G2_BN, AFD_NF_G2_ST, false> {};
+template <>
+struct GemmPair<true, kWide>
+    : GemmPairT<AFD_WF_G1_BN, AFD_WF_G1_ST, AFD_WF_G2_BN, AFD_WF_G2_ST, false, 0, AFD_WIDE_PAIR> {};
+template <>
+struct GemmPair<true, kWideSingle> : GemmPairT<128, 4, 128, 4, false> {};
 
 // Token-tile TMA box height of the gate/up (gemm = 1) or down (gemm = 2) kernel of a shape.
-template <bool NARROW>
+template <int SHAPE>
 uint32_t box_rows(bool fp8, int gemm) {
   if (fp8) {
-    using P = GemmPair<true, NARROW>;
-    return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, false, 1>::kBoxRows;
+    using P = GemmPair<true, SHAPE>;
+    return gemm == 1 ? GemmShape<P::bn1, false, 0, P::pair>::kBoxRows : GemmShape<P::bn2, false, 1, P::pair>::kBoxRows;
   }
-  using P = GemmPair<false, NARROW>;
-  return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, P::split, 1>::kBoxRows;
+  using P = GemmPair<false, SHAPE>;
+  return gemm == 1 ? GemmShape<P::bn1, false, 0, P::pair>::kBoxRows
+                   : GemmShape<P::bn2, P::split, 1, P::pair>::kBoxRows;
 }
 
-template <bool FP8, bool NARROW>
+// both wide shapes load token tiles through the same tensor maps, so their boxes must agree
+template <bool FP8>
+constexpr bool wide_boxes_agree() {
+  using A = GemmPair<FP8, kWide>;
+  using B = GemmPair<FP8, kWideSingle>;
+  return GemmShape<A::bn1, false, 0, A::pair>::kBoxRows == GemmShape<B::bn1, false, 0, B::pair>::kBoxRows &&
+         GemmShape<A::bn2, A::split, 1, A::pair>::kBoxRows == GemmShape<B::bn2, B::split, 1, B::pair>::kBoxRows;
+}
+static_assert(wide_boxes_agree<false>() && wide_boxes_agree<true>(), "wide token-tile boxes");
+
+template <bool FP8, int SHAPE>
 cudaError_t set_pair_attrs() {
-  using P = GemmPair<FP8, NARROW>;
+  using P = GemmPair<FP8, SHAPE>;
   if constexpr (P::fused) {
     return set_gemm_attr<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>();
   } else {
-    cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false>();
+    cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false, P::pair>();
     if (e != cudaSuccess) return e;
-    return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split>();
+    return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split, P::pair>();
   }
 }
 
 template <bool FP8>
 cudaError_t set_all_gemm_attrs() {
-  cudaError_t e = set_pair_attrs<FP8, true>();
+  cudaError_t e = set_pair_attrs<FP8, kNarrow>();
   if (e != cudaSuccess) return e;
   e = set_gemm_attr<kRouterBN, kRouterStages, false, 2, false>();
   if (e != cudaSuccess) return e;
-  return set_pair_attrs<FP8, false>();
+  e = set_pair_attrs<FP8, kWide>();
+  if (e != cudaSuccess) return e;
+  return set_pair_attrs<FP8, kWideSingle>();
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false>
 void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
                  const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
-  grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
-      a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
+  if constexpr (PAIR) {
+    // clusters of two CTAs (grid even); the launch error, if any, surfaces through the
+    // cudaGetLastError check that ends the stage
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid & ~1));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = gemm_smem_bytes<BN, ST, SPLIT, MODE, PAIR>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>, a, b, a2 ? *a2 : a, b2 ? *b2 : b,
+                       args);
+  } else {
+    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
+        a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
+  }
+}
+
+// CTAs of a CTA-pair GEMM launch: every pair of the persistent grid resident at once (two SMs
+// of a TPC each), so no pair waits for another to finish its share of the units.
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
+int pair_grid_for(int num_sms) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_smem_bytes<BN, ST, SPLIT, MODE, true>();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, true>, &cfg) !=
+          cudaSuccess ||
+      clusters <= 0) {
+    cudaGetLastError();  // clear; fall back to one pair per two SMs
+    return num_sms & ~1;
+  }
+  return std::min(num_sms & ~1, 2 * clusters);
+}
+
+template <bool FP8>
+int pair_grid(int num_sms) {
+  using P = GemmPair<FP8, kWide>;
+  if constexpr (!P::pair) {
+    return num_sms;
+  } else {
+    return std::min(pair_grid_for<P::bn1, P::st1, FP8, 0, false>(num_sms),
+                    pair_grid_for<P::bn2, P::st2, FP8, 1, P::split>(num_sms));
+  }
 }
 
 // K split of the tensor-core router: enough units to cover the SMs, every split non-empty.
@@ -363,10 +451,11 @@ int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T
   return AFD_OK;
 }
 
-template <bool FP8, bool NARROW>
+template <bool FP8, int SHAPE>
 void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
-  using P = GemmPair<FP8, NARROW>;
-  const int shape = NARROW ? 0 : 1;
+  using P = GemmPair<FP8, SHAPE>;
+  constexpr bool NARROW = SHAPE == kNarrow;
+  const int shape = NARROW ? 0 : 1;  // token-row tensor maps: both wide shapes use 64-row boxes
   const afd_ffn_cfg& c = h->cfg;
   const int R = T * c.k + T;
   GemmArgs g1{};
@@ -377,7 +466,7 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g1.G = h->G;
   g1.K = c.H;
   g1.a_rows = 2 * c.I;
-  g1.mt_stride = 128;
+  g1.mt_stride = P::gate_rows_per_unit;
   g1.second_off = c.I;
   g1.out = h->act;
   g1.out_ld = c.I;
@@ -408,7 +497,8 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
     return;
   }
   record(h, 5, s);
-  launch_gemm<P::bn1, P::st1, FP8, 0, false>(h->num_sms, h->tm_w13, h->tm_xp[shape], g1, s);
+  const int grid = P::pair ? h->pair_grid : h->num_sms;
+  launch_gemm<P::bn1, P::st1, FP8, 0, false, P::pair>(grid, h->tm_w13, h->tm_xp[shape], g1, s);
   record(h, 6, s);
   if (FP8)
     quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
@@ -417,36 +507,47 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g2.K = c.I;
   g2.a_rows = c.H;
   g2.mt_stride = 256;
-  g2.second_off = 128;
+  g2.second_off = P::pair ? 0 : 128;  // a pair's down unit is one 256-row tile (128 rows per CTA)
   g2.out = h->Y;
   g2.out_ld = c.H;
   g2.a_scale = h->w.w2_scale;
   g2.b_scale = h->ascale;
   record(h, 7, s);
-  launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(h->num_sms, h->tm_w2, h->tm_act[shape], g2, s);
+  launch_gemm<P::bn2, P::st2, FP8, 1, P::split, P::pair>(grid, h->tm_w2, h->tm_act[shape], g2, s);
 }
 
 int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   const bool narrow = use_narrow(h, T);
-  int bn1, bn2;
+  const int shape = narrow ? kNarrow : (c.I % 256 == 0 ? kWide : kWideSingle);
+  int bn1, bn2, gate_rows;
+  auto pick = [&](auto p) {
+    using P = decltype(p);
+    bn1 = P::bn1;
+    bn2 = P::bn2;
+    gate_rows = P::gate_rows_per_unit;
+  };
   if (h->fp8) {
-    bn1 = narrow ? GemmPair<true, true>::bn1 : GemmPair<true, false>::bn1;
-    bn2 = narrow ? GemmPair<true, true>::bn2 : GemmPair<true, false>::bn2;
+    if (shape == kNarrow) pick(GemmPair<true, kNarrow>{});
+    else if (shape == kWide) pick(GemmPair<true, kWide>{});
+    else pick(GemmPair<true, kWideSingle>{});
   } else {
-    bn1 = narrow ? GemmPair<false, true>::bn1 : GemmPair<false, false>::bn1;
-    bn2 = narrow ? GemmPair<false, true>::bn2 : GemmPair<false, false>::bn2;
+    if (shape == kNarrow) pick(GemmPair<false, kNarrow>{});
+    else if (shape == kWide) pick(GemmPair<false, kWide>{});
+    else pick(GemmPair<false, kWideSingle>{});
   }
   record(h, 4, s);
-  build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn1, bn2, c.I / 128, c.H / 256,
+  build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn1, bn2, c.I / gate_rows, c.H / 256,
                                           h->grp_rows, h->grp_base, h->ub1, h->ub2, h->tile_base, h->tile_done,
                                           h->err);
   if (h->fp8) {
-    if (narrow) run_gemms<true, true>(h, T, s);
-    else run_gemms<true, false>(h, T, s);
+    if (shape == kNarrow) run_gemms<true, kNarrow>(h, T, s);
+    else if (shape == kWide) run_gemms<true, kWide>(h, T, s);
+    else run_gemms<true, kWideSingle>(h, T, s);
   } else {
-    if (narrow) run_gemms<false, true>(h, T, s);
-    else run_gemms<false, false>(h, T, s);
+    if (shape == kNarrow) run_gemms<false, kNarrow>(h, T, s);
+    else if (shape == kWide) run_gemms<false, kWide>(h, T, s);
+    else run_gemms<false, kWideSingle>(h, T, s);
   }
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
@@ -604,8 +705,9 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   // token-row maps: box heights must match GemmShape<...>::kBoxRows of the kernels using them
   const void* act_src = h->fp8 ? static_cast<const void*>(h->actq) : h->act;
   const uint64_t act_rows = h->fp8 ? R : 2 * R;
-  const uint32_t box_xp[2] = {box_rows<true>(h->fp8, 1), box_rows<false>(h->fp8, 1)};
-  const uint32_t box_act[2] = {box_rows<true>(h->fp8, 2), box_rows<false>(h->fp8, 2)};
+  const uint32_t box_xp[2] = {box_rows<kNarrow>(h->fp8, 1), box_rows<kWide>(h->fp8, 1)};
+  const uint32_t box_act[2] = {box_rows<kNarrow>(h->fp8, 2), box_rows<kWide>(h->fp8, 2)};
+
   bool ok = encode_2d(&h->tm_w13, weights->w13, h->fp8, c.H, G * 2 * c.I, 128) &&
             encode_2d(&h->tm_w2, weights->w2, h->fp8, c.I, G * c.H, 128) &&
             encode_2d(&h->tm_xp[0], h->xp, h->fp8, c.H, R, box_xp[0]) &&
@@ -616,6 +718,8 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
   if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  h->pair_grid = h->fp8 ? pair_grid<true>(h->num_sms) : pair_grid<false>(h->num_sms);
+  if (h->pair_grid < 2) { cudaFree(h->ws); delete h; return AFD_ERR_UNSUPPORTED; }
   router_split_planes_kernel<<<256, 256>>>(weights->router_w, static_cast<size_t>(c.E) * c.H,
                                            static_cast<__nv_bfloat16*>(h->wr_planes));
   e = cudaGetLastError();

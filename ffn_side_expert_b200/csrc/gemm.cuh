@@ -88,14 +88,19 @@ struct GemmArgs {
   int mt1;                   // gate/up units per N tile (I / 128)
 };
 
-template <int BN, bool SPLIT_B = false, int MODE = 0>
+// PAIR: a CTA pair (2-CTA cluster) shares each unit through M = 256 pair MMAs; every CTA holds
+// 128 rows of each weight tile and half of the token tile (BN / 2 rows).  Gate/up units cover
+// 256 gate rows and the 256 matching up rows (two accumulators), down units 256 output rows
+// (one accumulator).
+template <int BN, bool SPLIT_B = false, int MODE = 0, bool PAIR = false>
 struct GemmShape {
   static constexpr bool kFused = MODE == 3;
-  static constexpr int kNA = MODE == 2 ? 3 : 2;         // weight tiles per stage
-  static constexpr int kNDU = MODE == 2 ? 1 : 2;        // accumulators per unit
+  static constexpr int kNA = MODE == 2 ? 3 : (PAIR && MODE == 1 ? 1 : 2);   // weight tiles per stage
+  static constexpr int kNDU = MODE == 2 ? 1 : (PAIR && MODE == 1 ? 1 : 2);  // accumulators per unit
   static constexpr int kATile = 128 * 128;              // one 128-row x 128-byte weight tile
   static constexpr int kAStage = kNA * kATile;
-  static constexpr int kBTile = BN * 128;               // up to BN token rows x 128 bytes
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;     // token rows of this CTA's tile
+  static constexpr int kBTile = kBRows * 128;           // up to kBRows token rows x 128 bytes
   static constexpr int kBStage = (SPLIT_B ? 2 : 1) * kBTile;
   static constexpr int kStageBytes = kAStage + kBStage;
   // two-term activations in one MMA (hi rows, then lo rows): the N of an MMA doubles
@@ -107,7 +112,7 @@ struct GemmShape {
   // becoming the bottleneck; a box may overrun the unit's rows (the MMA reads only n16 rows)
   // except in the concatenated layout, where the lo rows follow the hi rows directly.
   // kBoxRowsX: single-plane token tiles (the gate/up side of the fused kernel)
-  static constexpr int kBoxRowsX = BN < 64 ? BN : 64;
+  static constexpr int kBoxRowsX = kBRows < 64 ? kBRows : 64;
   static constexpr int kBoxRows = kConcat ? (BN <= 32 ? 16 : 32) : kBoxRowsX;
   // concatenated layout: hi rows padded to whole boxes, then the lo rows
   __device__ static int npad(int n16) { return kConcat ? (n16 + kBoxRows - 1) / kBoxRows * kBoxRows : n16; }
@@ -118,6 +123,7 @@ struct GemmShape {
                                    : kColsUsed <= 256 ? 256 : 512;
   static_assert(kColsUsed <= 512, "TMEM has 512 columns");
   static_assert(BN % 16 == 0 && BN <= 256, "N tile");
+  static_assert(!PAIR || ((MODE == 0 || MODE == 1) && !kConcat), "pairs serve the wide gate/up and down GEMMs");
   static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 };
 
@@ -126,10 +132,10 @@ struct GemmShape {
 constexpr int kMaxGroups = 257;
 constexpr int kSchedBytes = (kMaxGroups + 1) * 16;
 
-template <int BN, int STAGES, bool SPLIT_B, int MODE = 0>
+template <int BN, int STAGES, bool SPLIT_B, int MODE = 0, bool PAIR = false>
 constexpr int gemm_smem_bytes() {
   return (MODE == 3 ? 2 : 1) * kSchedBytes + 1024 /*alignment slack*/ +
-         STAGES * GemmShape<BN, SPLIT_B, MODE>::kStageBytes + 256 /*barriers*/;
+         STAGES * GemmShape<BN, SPLIT_B, MODE, PAIR>::kStageBytes + 256 /*barriers*/;
 }
 
 // Largest g with tab[g].x (first unit of group g) <= u; the table sits in shared memory.
@@ -223,14 +229,14 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
   return true;
 }
 
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs args) {
   static_assert(!(SPLIT_B && (FP8 || (MODE != 1 && MODE != 3))), "two-term B only for the bf16 down GEMM");
   static_assert(!((MODE == 2 || MODE == 3) && FP8), "router and fused modes run on bf16");
-  using S = GemmShape<BN, SPLIT_B, MODE>;
+  using S = GemmShape<BN, SPLIT_B, MODE, PAIR>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
 
@@ -255,6 +261,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pair: rank in the pair, the pair's index and count; the unit loop runs over pairs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -263,7 +274,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int i = 0; i < kNacc; ++i) {
       mbar_init(tfull + 8u * i, 1);
-      mbar_init(tempty + 8u * i, kEpiWarps);
+      mbar_init(tempty + 8u * i, (PAIR ? 2 : 1) * kEpiWarps);
     }
     mbar_init(done_bar, 1);
     for (int i = 0; i < kNacc; ++i) mbar_init(epi_bar + 8u * i, kEpiWarps);
@@ -277,8 +288,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), S::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (args.single_rows < 0) {
     for (int g = threadIdx.x; g <= args.G; g += blockDim.x) {
@@ -293,6 +309,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
   tc_fence_before();
   __syncthreads();
+  // the peer's barriers are initialised before any TMA or commit of the pair reaches them
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -307,18 +325,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t ph = 0;
     int issued = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+    // a pair's stages complete on the first CTA's full barriers (both halves counted there)
+    const uint32_t full_tx = PAIR ? mapa_shared(full, 0) : full;
+    for (int u = unit0; u < total && ok; u += unit_step) {
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       // the down side of the fused kernel uses the second set of maps and coordinates
       const bool down = MODE == 3 && w.mode == 1;
       const CUtensorMap* mA = down ? &tmA2 : &tmA;
       const CUtensorMap* mB = down ? &tmB2 : &tmB;
-      const int ya = down ? w.g * args.a_rows2 + w.mt * args.mt_stride2 : w.g * args.a_rows + w.mt * args.mt_stride;
+      const int ya = (down ? w.g * args.a_rows2 + w.mt * args.mt_stride2 : w.g * args.a_rows + w.mt * args.mt_stride) +
+                     (PAIR ? 128 * static_cast<int>(rank) : 0);
       const int soff = down ? args.second_off2 : args.second_off;
       const bool two = SPLIT_B && (MODE != 3 || down);           // hi and lo planes
       const int boxr = (MODE == 3 && !down) ? S::kBoxRowsX : S::kBoxRows;
-      const int nbox = (w.n16 + boxr - 1) / boxr;                  // token-tile boxes per plane
-      const uint32_t tx = S::kAStage + (two ? 2u : 1u) * static_cast<uint32_t>(nbox * boxr) * 128u;
+      // this CTA's token rows: all n16 rows, or its half of them in a pair
+      const int brows = PAIR ? w.n16 / 2 : w.n16;
+      const int brow0 = w.row0 + (PAIR ? static_cast<int>(rank) * brows : 0);
+      const int nbox = (brows + boxr - 1) / boxr;                  // token-tile boxes per plane
+      const uint32_t tx = (PAIR ? 2u : 1u) *
+                          (S::kAStage + (two ? 2u : 1u) * static_cast<uint32_t>(nbox * boxr) * 128u);
       // the lo activation rows follow the (padded) hi rows or sit one tile further
       const uint32_t lo_off = S::kConcat ? static_cast<uint32_t>(S::npad(w.n16)) * 128u : S::kBTile;
       const uint64_t apol = MODE == 2 ? kEvictLast : args.a_policy;
@@ -326,44 +351,57 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int kc = w.kc0; kc < w.kc1; ++kc) {
         if (!mbar_wait(empty + 8u * s, ph ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t st = base + s * S::kStageBytes;
-        const uint32_t fb = full + 8u * s;
+        const uint32_t fb = full_tx + 8u * s;
         const int x = kc * kKChunk;
-        mbar_arrive_expect_tx(fb, tx);
-        // the pair (MODE 0/1) or the three router planes (MODE 2), second_off apart
+        if (leader) mbar_arrive_expect_tx(full + 8u * s, tx);
+        // the tile pair (MODE 0/1), one tile (pair down), or the three router planes (MODE 2)
 #pragma unroll
-        for (int i = 0; i < S::kNA; ++i)
-          tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
+        for (int i = 0; i < S::kNA; ++i) {
+          if constexpr (PAIR) tma_load_2d_pair(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
+          else tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
+        }
         const uint32_t sb = st + S::kAStage;
-        for (int b = 0; b < nbox; ++b)
-          tma_load_2d(sb + b * boxr * 128, mB, fb, x, w.row0 + b * boxr, kEvictLast);
+        for (int b = 0; b < nbox; ++b) {
+          if constexpr (PAIR) tma_load_2d_pair(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
+          else tma_load_2d(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
+        }
         if (two) {
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sb + lo_off + b * boxr * 128, mB, fb, x, args.lo_rows + w.row0 + b * boxr, kEvictLast);
+          for (int b = 0; b < nbox; ++b) {
+            const int y = args.lo_rows + brow0 + b * boxr;
+            if constexpr (PAIR) tma_load_2d_pair(sb + lo_off + b * boxr * 128, mB, fb, x, y, kEvictLast);
+            else tma_load_2d(sb + lo_off + b * boxr * 128, mB, fb, x, y, kEvictLast);
+          }
         }
         ++issued;
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
     if (!ok) { *abort_flag = 1; atomicOr(args.err, kErrTimeout); }
-    // drain: the last min(issued, STAGES) stages may still be landing in shared memory
+    // drain: the last min(issued, STAGES) stages may still be landing in shared memory.  The
+    // second CTA of a pair cannot see its loads land (they count on the first CTA's barrier);
+    // it waits until the pair's MMAs have consumed them instead (bounded either way).
     for (int i = 0; i < min(issued, STAGES); ++i) {
       if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
       volatile int never = 0;
-      mbar_wait(full + 8u * s, ph, &never);
+      mbar_wait((leader ? full : empty) + 8u * s, ph, &never);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ---------------------------------------------------------------- MMA issuer
+    // (in a pair, the first CTA issues the pair's MMAs; its commits reach both CTAs)
     int s = 0;
     uint32_t ph = 0;
     int acc = 0;
     uint32_t acc_ph = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+    for (int u = unit0; u < total && ok; u += unit_step) {
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
       const bool cat = S::kConcat && down;
-      const uint32_t idesc = idesc_m128(cat ? 2 * S::npad(w.n16) : w.n16, FP8);
-      if (!mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
+      const uint32_t idesc = idesc_mn(PAIR ? 256 : 128, cat ? 2 * S::npad(w.n16) : w.n16, FP8);
+      // (a pair's accumulators are released by the epilogue warps of both CTAs)
+      const bool freed = PAIR ? mbar_wait_cluster(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)
+                              : mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag);
+      if (!freed) { ok = false; break; }
       tc_fence_after();
       const uint32_t d0 = tmem + static_cast<uint32_t>(acc * S::kUnitCols);
       const uint32_t d1 = d0 + S::kUnitCols / 2;
@@ -382,6 +420,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_mma<false>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             tc_mma<false>(d0, da1 + 2 * kk, db + 2 * kk, idesc, 1u);
             tc_mma<false>(d0, da2 + 2 * kk, db + 2 * kk, idesc, 1u);
+          } else if constexpr (PAIR) {
+            // gate/up: the 256 gate rows and the 256 up rows; down: 256 output rows (+ lo plane)
+            tc_mma_pair<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+            if constexpr (S::kNDU == 2) tc_mma_pair<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+            if constexpr (SPLIT_B) {
+              const uint64_t dl = sw128_desc(st + S::kAStage + S::kBTile);
+              tc_mma_pair<FP8>(d0, da0 + 2 * kk, dl + 2 * kk, idesc, 1u);
+            }
           } else {
             tc_mma<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
@@ -394,16 +440,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
           }
         }
-        tc_commit(empty + 8u * s);  // frees the stage once these MMAs have read it
+        // frees the stage (in both CTAs of a pair) once these MMAs have read it
+        if constexpr (PAIR) tc_commit_pair_mc(empty + 8u * s, 0x3);
+        else tc_commit(empty + 8u * s);
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
-      tc_commit(tfull + 8u * acc);
+      if constexpr (PAIR) tc_commit_pair_mc(tfull + 8u * acc, 0x3);
+      else tc_commit(tfull + 8u * acc);
       if (++acc == kNacc) { acc = 0; acc_ph ^= 1u; }
     }
     if (!ok) { *abort_flag = 1; atomicOr(args.err, kErrTimeout); }
     // every MMA issued above has completed once this commit arrives
-    tc_commit(done_bar);
+    if constexpr (PAIR) tc_commit_pair(done_bar);
+    else tc_commit(done_bar);
     volatile int never = 0;
     mbar_wait(done_bar, 0, &never);
   } else if (warp >= 2 && warp < 2 + kEpiWarps) {
@@ -415,7 +465,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     int acc = 0;
     uint32_t acc_ph = 0;
     uint32_t epi_ph = 0;  // parity bit per accumulator buffer
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    // a pair's epilogue warps release an accumulator on the first CTA's barrier
+    const uint32_t tempty_rel = PAIR ? mapa_shared(tempty, 0) : tempty;
+    for (int u = unit0; u < total; u += unit_step) {
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       if (!mbar_wait(tfull + 8u * acc, acc_ph, abort_flag)) {
         *abort_flag = 1;
@@ -427,7 +479,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t t1 = t0 + S::kUnitCols / 2;
       // weight rows of this thread in the two tiles
       const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
-      const int wrow0 = w.mt * (MODE == 3 && down ? args.mt_stride2 : args.mt_stride) + m;
+      const int wrow0 = w.mt * (MODE == 3 && down ? args.mt_stride2 : args.mt_stride) +
+                        (PAIR ? 128 * static_cast<int>(rank) : 0) + m;
       const int wrow1 = wrow0 + (MODE == 3 && down ? args.second_off2 : args.second_off);
       if constexpr (MODE == 2) {  // partial logits [split][t][e]; rows past E are padding
         const int e = wrow0;
@@ -457,8 +510,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
           uint32_t r0[16], r1[16];
           tmem_ld16(t0 + c, r0);
-          tmem_ld16(t1 + c, r1);
-          tmem_ld_wait(r0, r1);
+          if constexpr (S::kNDU == 2) {
+            tmem_ld16(t1 + c, r1);
+            tmem_ld_wait(r0, r1);
+          } else {
+            tmem_ld_wait(r0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r1[i] = 0u;
+          }
           if (S::kConcat && down) {  // add the lo-plane half (columns npad..) of each tile
             uint32_t l0[16], l1[16];
             tmem_ld16(t0 + S::npad(w.n16) + c, l0);
@@ -497,12 +556,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               } else if constexpr (FP8) {  // W8A8: expert outputs kept as bf16 (combine input)
                 __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.out) + row * args.out_ld;
                 y[wrow0] = __float2bfloat16_rn(v0);
-                y[wrow1] = __float2bfloat16_rn(v1);
+                if constexpr (S::kNDU == 2) y[wrow1] = __float2bfloat16_rn(v1);
               } else {
                 float* y = static_cast<float*>(MODE == 3 ? args.out2 : args.out) +
                            row * (MODE == 3 ? args.out_ld2 : args.out_ld);
                 y[wrow0] = v0;
-                y[wrow1] = v1;
+                if constexpr (S::kNDU == 2) y[wrow1] = v1;
               }
             }
           }
@@ -528,16 +587,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           epi_ph ^= 1u << acc;
         }
       }
-      if (lane == 0) mbar_arrive(tempty + 8u * acc);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(tempty_rel + 8u * acc);
+        else mbar_arrive(tempty + 8u * acc);
+      }
       if (++acc == kNacc) { acc = 0; acc_ph ^= 1u; }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still signal its barriers
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, S::kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, S::kTmemCols);
+    else tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 
