@@ -38,15 +38,39 @@ combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int3
   const YT* ys = Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
   for (int v = threadIdx.x; v < H / 4; v += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const int p = sp[j];
-      if (p < 0) continue;
-      const float wj = sw[j];
-      const float4 y = load4(Y + static_cast<size_t>(p) * H, v);
-      acc.x = fmaf(wj, y.x, acc.x);
-      acc.y = fmaf(wj, y.y, acc.y);
-      acc.z = fmaf(wj, y.z, acc.z);
-      acc.w = fmaf(wj, y.w, acc.w);
+    if constexpr (sizeof(YT) == 4) {
+      // fp32 rows: four rows' loads in flight at once, accumulated in j order (measured 15 %
+      // faster at T=256; the bf16 rows of the W8A8 path run faster with the plain loop)
+      for (int j0 = 0; j0 < k; j0 += 4) {
+        float4 y[4];
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+          const int j = j0 + d;
+          const int p = j < k ? sp[j] : -1;
+          y[d] = p >= 0 ? load4(Y + static_cast<size_t>(p) * H, v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+          const int j = j0 + d;
+          if (j >= k || sp[j] < 0) continue;
+          const float wj = sw[j];
+          acc.x = fmaf(wj, y[d].x, acc.x);
+          acc.y = fmaf(wj, y[d].y, acc.y);
+          acc.z = fmaf(wj, y[d].z, acc.z);
+          acc.w = fmaf(wj, y[d].w, acc.w);
+        }
+      }
+    } else {
+      for (int j = 0; j < k; ++j) {
+        const int p = sp[j];
+        if (p < 0) continue;
+        const float wj = sw[j];
+        const float4 y = load4(Y + static_cast<size_t>(p) * H, v);
+        acc.x = fmaf(wj, y.x, acc.x);
+        acc.y = fmaf(wj, y.y, acc.y);
+        acc.z = fmaf(wj, y.z, acc.z);
+        acc.w = fmaf(wj, y.w, acc.w);
+      }
     }
     if (with_shared) {
       const float4 s = load4(ys, v);

@@ -101,16 +101,26 @@ router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __re
   if (t >= T) return;
   float v[8];
   unsigned taken = 0;
+  // partial logits summed in split order; the eight loads of one split are independent, so a
+  // lane waits for one memory round trip per split rather than one per (split, value)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const float* ps = part + (static_cast<size_t>(sp) * T + t) * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) v[i] += ps[e];
+    }
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
-    float s = -INFINITY;
     if (e < E) {
-      s = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) s += part[(static_cast<size_t>(sp) * T + t) * E + e];
-      if (bias) s += bias[e];
+      if (bias) v[i] += bias[e];
+    } else {
+      v[i] = -INFINITY;
     }
-    v[i] = s;
   }
   int my_e = -1;
   float my_v = -INFINITY;
