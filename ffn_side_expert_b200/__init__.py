@@ -167,7 +167,8 @@ def afd_ffn_forward_host_batches(h, hidden_host_list, out_host_list, T, stream=N
 
 
 def afd_ffn_set_stage_events(h, events) -> int:
-    """events: sequence of torch.cuda.Event (AFD_FFN_NUM_STAGES + 1 of them) or None.
+    """events: sequence of torch.cuda.Event or None entries (AFD_FFN_NUM_STAGES + 1 of them; a
+    None entry skips that stage boundary), or None to turn stage events off.
 
     torch creates an event's CUDA handle at its first record; events not yet created are
     recorded once on the current stream here so that the library receives real handles.
@@ -175,9 +176,9 @@ def afd_ffn_set_stage_events(h, events) -> int:
     if not events:
         return _lib.afd_ffn_set_stage_events(h, None, 0)
     for e in events:
-        if not e.cuda_event:
+        if e is not None and not e.cuda_event:
             e.record()
-    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event if e is not None else None for e in events])
     return _lib.afd_ffn_set_stage_events(h, arr, len(events))
 
 

@@ -395,7 +395,7 @@ void router_ksplit(int T, int H, int E, int sms, int* ksplit, int* kc_per) {
 
 void record(afd_ffn_handle* h, int stage, cudaStream_t s) {
   // a failure here surfaces through the cudaGetLastError check that ends each stage
-  if (h->n_events > stage) cudaEventRecord(h->events[stage], s);
+  if (h->n_events > stage && h->events[stage]) cudaEventRecord(h->events[stage], s);
 }
 
 // ------------------------------------------------------------------ stages
@@ -884,9 +884,7 @@ int afd_ffn_forward_host_batches(afd_ffn_handle* h, const void* const* hidden_ho
 int afd_ffn_set_stage_events(afd_ffn_handle* h, void* const* events, int32_t n_events) {
   if (!h || n_events < 0 || n_events > AFD_FFN_NUM_STAGES + 1) return AFD_ERR_INVALID_ARG;
   if (n_events > 0 && !events) return AFD_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i)
-    if (!events[i]) return AFD_ERR_INVALID_ARG;
-  for (int i = 0; i < n_events; ++i) h->events[i] = static_cast<cudaEvent_t>(events[i]);
+  for (int i = 0; i < n_events; ++i) h->events[i] = static_cast<cudaEvent_t>(events[i]);  // NULL: skipped
   h->n_events = n_events;
   return AFD_OK;
 }

@@ -143,8 +143,9 @@ int afd_ffn_forward_host_batches(afd_ffn_handle *h, const void *const *hidden_ho
  * afd_ffn_forward records on its stream before each stage and after the last one.  Stages,
  * in order: router logits, top-k, dispatch order, row gather, GEMM schedule, gate/up GEMM,
  * activation quantisation (W8A8 only; empty otherwise), down GEMM, combine -- so
- * AFD_FFN_NUM_STAGES + 1 events, each already created (non-NULL; AFD_ERR_INVALID_ARG otherwise).
- * n_events = 0 (events NULL) turns it off. */
+ * AFD_FFN_NUM_STAGES + 1 events, each already created.  A NULL entry skips that boundary (a
+ * caller timing one stage passes only the two events around it, so the others add nothing to
+ * the stream).  n_events = 0 (events NULL) turns it off. */
 #define AFD_FFN_NUM_STAGES 9
 int afd_ffn_set_stage_events(afd_ffn_handle *h, void *const *events, int32_t n_events);
 

@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 import torch
 
+import ffn_side_expert_b200 as afd
 import synth
 from layer_support import BF16_TOL, W_TOL, Layer, rel_max_err, to64
 from oracle import moe
@@ -122,3 +123,19 @@ def test_cuda_graph_replay(layer):
     torch.cuda.synchronize()
     assert torch.equal(out, eager)
     del g
+
+
+def test_sparse_stage_events(layer):
+    # only the boundaries around stage 5 (the expert GEMMs) are recorded; the others are NULL
+    eager = layer.forward().clone()
+    n = afd.AFD_FFN_NUM_STAGES + 1
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    events = [e0 if s == 5 else e1 if s == 6 else None for s in range(n)]
+    layer.mod.set_stage_events(events)
+    out = layer.forward()
+    layer.mod.set_stage_events(None)
+    torch.cuda.synchronize()
+    assert e0.elapsed_time(e1) > 0.0
+    assert torch.equal(out, eager)
+    assert layer.mod.get_error() == 0
