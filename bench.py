@@ -36,13 +36,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
 # of the decode shape, from a one-pass ncu capture of two launches at T=256, H=7168, E=256,
-# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 068 632 320 and
-# 23 060 022 272 bytes for 257 touched experts.  Traffic grows with the experts whose weights
+# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 054 580 736 and
+# 23 121 128 448 bytes for 257 touched experts.  Traffic grows with the experts whose weights
 # are streamed, and it is reported only while the kernel source and its instantiation are the
 # ones that were captured.
 MEASURED_TRAFFIC = {
-    "sources_sha256": "3b01a3473e3a27d2e5c30d7711436fc452ca3def330c9ffc2a194d9ac53678cf",
-    "bytes_per_touched_expert": (23068632320 + 23060022272) / 2 / 257,
+    "sources_sha256": "a4ad12a3240a562c7d0eba40359ef585bda779308149208138a0b0964c545765",
+    "bytes_per_touched_expert": (23054580736 + 23121128448) / 2 / 257,
 }
 METRIC = "MoE-FFN tokens/s/layer"
 

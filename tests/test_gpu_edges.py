@@ -150,6 +150,19 @@ def test_wide_tiles_single_cta_when_i_is_not_a_multiple_of_256(dtype):
         L.close()
 
 
+@pytest.mark.parametrize("T", [40, 200])
+def test_largest_top_k(T):
+    # k = 32, the largest top-k the library takes: a full warp of selections per token, 1024
+    # threads per CTA in the gate-weight refinement, 33 destinations per dispatched token.
+    # T=40 runs the decode tiles (fused kernel), T=200 the wide ones.
+    cfg = synth.MoEConfig("k32", T=200, H=256, E=64, k=32, I=256, S=1, seed=28)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, T)
+    finally:
+        L.close()
+
+
 @pytest.mark.parametrize("T", [64, 23])
 def test_w8a8_small(T):
     cfg = synth.MoEConfig("fp8s", T=64, H=512, E=8, k=2, I=256, S=1, dtype="fp8", seed=25)
