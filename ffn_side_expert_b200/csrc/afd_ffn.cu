@@ -81,6 +81,10 @@ struct afd_ffn_handle {
   cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
 
   CUtensorMap tm_w13, tm_w2, tm_wr;
+  // bf16 large micro-batches: f16 copy of W2 and the f16 activation plane (single-term down GEMM)
+  void* w2h = nullptr;       // [E+S][H][I] f16, owned; NULL when unused
+  bool act16 = false;
+  CUtensorMap tm_w2h, tm_act16;
   CUtensorMap tm_xp[2], tm_act[2];  // token rows for the [narrow, wide] shapes (box heights differ)
   cudaStream_t last_stream = nullptr;
   int last_cuda_error = 0;
@@ -159,12 +163,24 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false, bool ACT16 = false>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR, ACT16>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               gemm_smem_bytes<BN, ST, SPLIT, MODE, PAIR>());
 }
+
+// bf16 large micro-batches with f16 activations: gate/up (f16 act plane) and down (f16 operands)
+#ifndef AFD_ACT16
+#define AFD_ACT16 1
+#endif
+#ifndef AFD_ACT16_G1_ST
+#define AFD_ACT16_G1_ST 4
+#endif
+#ifndef AFD_ACT16_G2_ST
+#define AFD_ACT16_G2_ST 4
+#endif
+constexpr int kAct16BN = 128;
 
 // (gate/up, down) kernel pairs of each path and tile shape: N tile and ring stages of each
 // GEMM.  Compile-time tunable for tile sweeps: -DAFD_<path>_BN=.. -DAFD_<path>_ST=..
@@ -319,10 +335,17 @@ cudaError_t set_all_gemm_attrs() {
   if (e != cudaSuccess) return e;
   e = set_pair_attrs<FP8, kWide>();
   if (e != cudaSuccess) return e;
-  return set_pair_attrs<FP8, kWideSingle>();
+  e = set_pair_attrs<FP8, kWideSingle>();
+  if (e != cudaSuccess) return e;
+  if constexpr (!FP8) {
+    e = set_gemm_attr<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, false, true>();
+    if (e != cudaSuccess) return e;
+    e = set_gemm_attr<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, false, true>();
+  }
+  return e;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false, bool ACT16 = false>
 void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
                  const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
   if constexpr (PAIR) {
@@ -343,8 +366,8 @@ void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const Gem
     cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>, a, b, a2 ? *a2 : a, b2 ? *b2 : b,
                        args);
   } else {
-    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT><<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(
-        a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
+    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, false, ACT16>
+        <<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
   }
 }
 
@@ -495,6 +518,26 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
     record(h, 6, s);
     record(h, 7, s);
     return;
+  }
+  if constexpr (!FP8 && !NARROW) {
+    if (h->act16 && !P::pair) {  // single-term down GEMM on f16 activations and the f16 copy of W2
+      GemmArgs a1 = g1;
+      a1.mt_stride = 128;
+      record(h, 5, s);
+      launch_gemm<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, false, true>(h->num_sms, h->tm_w13, h->tm_xp[1], a1, s);
+      record(h, 6, s);
+      GemmArgs a2 = a1;
+      a2.unit_base = h->ub2;
+      a2.K = c.I;
+      a2.a_rows = c.H;
+      a2.mt_stride = 256;
+      a2.second_off = 128;
+      a2.out = h->Y;
+      a2.out_ld = c.H;
+      record(h, 7, s);
+      launch_gemm<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, false, true>(h->num_sms, h->tm_w2h, h->tm_act16, a2, s);
+      return;
+    }
   }
   record(h, 5, s);
   const int grid = P::pair ? h->pair_grid : h->num_sms;
@@ -716,6 +759,27 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
             encode_2d(&h->tm_act[1], act_src, h->fp8, c.I, act_rows, box_act[1]) &&
             encode_2d(&h->tm_wr, h->wr_planes, false, c.H, 3 * static_cast<uint64_t>(c.E), 128);
   if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
+  // bf16 handles that can see large micro-batches keep an f16 copy of W2 for the single-term
+  // down GEMM (unless a weight exceeds the f16 range; then the two-term bf16 path stays)
+  if (AFD_ACT16 && !h->fp8 && static_cast<int64_t>(c.T_max) * c.k > 32 * static_cast<int64_t>(c.E)) {
+    const size_t n = G * c.H * static_cast<size_t>(c.I);
+    e = cudaMalloc(&h->w2h, n * 2);
+    if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+    bf16_to_f16_kernel<<<4 * h->num_sms, 256>>>(static_cast<const __nv_bfloat16*>(weights->w2),
+                                                static_cast<__half*>(h->w2h), n, h->err);
+    int overflow = 0;
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemcpy(&overflow, h->err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+    if (e != cudaSuccess) { cudaFree(h->w2h); cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+    h->act16 = overflow == 0 &&
+               encode_2d(&h->tm_w2h, h->w2h, false, c.I, G * c.H, 128) &&
+               encode_2d(&h->tm_act16, h->act, false, c.I, R, GemmShape<kAct16BN, false, 1>::kBoxRows);
+    if (!h->act16) {
+      cudaFree(h->w2h);
+      h->w2h = nullptr;
+    }
+  }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
   if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
   h->pair_grid = h->fp8 ? pair_grid<true>(h->num_sms) : pair_grid<false>(h->num_sms);
@@ -746,6 +810,7 @@ void afd_ffn_destroy(afd_ffn_handle* h) {
   }
   if (h->copy_in) cudaStreamDestroy(h->copy_in);
   if (h->copy_out) cudaStreamDestroy(h->copy_out);
+  if (h->w2h) cudaFree(h->w2h);
   cudaFree(h->ws);
   delete h;
 }

@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -83,6 +84,21 @@ combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int3
     packed.y = *reinterpret_cast<uint32_t*>(&hi);
     reinterpret_cast<uint2*>(out + static_cast<size_t>(t) * H)[v] = packed;
   }
+}
+
+// f16 copy of bf16 weights (the down projection of large bf16 micro-batches).  Every bf16 value
+// of magnitude in [2^-14, 65504] is exact in f16; smaller ones become f16 subnormals (absolute
+// error <= 2^-25); a magnitude above 65504 sets *overflow and the handle keeps the bf16 path.
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t n,
+                                   int* overflow) {
+  bool big = false;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float f = __bfloat162float(src[i]);
+    big |= !(fabsf(f) <= 65504.0f);  // also catches NaN
+    dst[i] = __float2half_rn(f);
+  }
+  if (big) atomicOr(overflow, 1);
 }
 
 // Widen bf16 rows to fp32 (copy-out of the W8A8 expert outputs by afd_ffn_expert_gemm).

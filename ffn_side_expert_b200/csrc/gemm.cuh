@@ -50,6 +50,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -229,13 +230,17 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
   return true;
 }
 
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool PAIR = false>
+// ACT16 (bf16 large micro-batches): the gate/up epilogue stores the SwiGLU output as one f16
+// plane (MODE 0), and the down GEMM multiplies it by an f16 copy of W2 (MODE 1, kind::f16 with
+// f16 operands) -- f16 keeps 10 mantissa bits where bf16 keeps 7, so one term suffices.
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool PAIR = false, bool ACT16 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs args) {
   static_assert(!(SPLIT_B && (FP8 || (MODE != 1 && MODE != 3))), "two-term B only for the bf16 down GEMM");
   static_assert(!((MODE == 2 || MODE == 3) && FP8), "router and fused modes run on bf16");
+  static_assert(!ACT16 || (!FP8 && !SPLIT_B && !PAIR && (MODE == 0 || MODE == 1)), "f16 activations: wide bf16 GEMMs");
   using S = GemmShape<BN, SPLIT_B, MODE, PAIR>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
@@ -397,7 +402,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
       const bool cat = S::kConcat && down;
-      const uint32_t idesc = idesc_mn(PAIR ? 256 : 128, cat ? 2 * S::npad(w.n16) : w.n16, FP8);
+      const uint32_t idesc = idesc_mn(PAIR ? 256 : 128, cat ? 2 * S::npad(w.n16) : w.n16, FP8, ACT16 && MODE == 1);
       // (a pair's accumulators are released by the epilogue warps of both CTAs)
       const bool freed = PAIR ? mbar_wait_cluster(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)
                               : mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag);
@@ -546,6 +551,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float act = silu_f(v0) * v1;  // gate tile first, up tile second
                 if constexpr (FP8) {
                   static_cast<float*>(args.out)[row * args.out_ld + wrow0] = act;
+                } else if constexpr (ACT16) {
+                  static_cast<__half*>(args.out)[row * args.out_ld + wrow0] = __float2half_rn(act);
                 } else {
                   const __nv_bfloat16 hi = __float2bfloat16_rn(act);
                   const __nv_bfloat16 lo = __float2bfloat16_rn(act - __bfloat162float(hi));

@@ -273,13 +273,14 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
 }
 
 // Instruction descriptor: fp32 accumulator, A and B K-major, M = m (128, or 256 for a CTA
-// pair), N = n (multiple of 16).  Operand format: bf16 (kind::f16) or e4m3 (kind::f8f6f4).
-__host__ __device__ constexpr uint32_t idesc_mn(int m, int n, bool fp8) {
-  return (1u << 4)                                   // D format f32
-         | ((fp8 ? 0u : 1u) << 7)                    // A format: e4m3 = 0, bf16 = 1
-         | ((fp8 ? 0u : 1u) << 10)                   // B format
-         | (static_cast<uint32_t>(n >> 3) << 17)     // N >> 3
-         | (static_cast<uint32_t>(m >> 4) << 24);    // M >> 4
+// pair), N = n (multiple of 16).  Operand format (A and B alike): bf16 or f16 (kind::f16: 1 =
+// bf16, 0 = f16) or e4m3 (kind::f8f6f4: 0).
+__host__ __device__ constexpr uint32_t idesc_mn(int m, int n, bool fp8, bool f16 = false) {
+  return (1u << 4)                                             // D format f32
+         | ((fp8 || f16 ? 0u : 1u) << 7)                       // A format
+         | ((fp8 || f16 ? 0u : 1u) << 10)                      // B format
+         | (static_cast<uint32_t>(n >> 3) << 17)               // N >> 3
+         | (static_cast<uint32_t>(m >> 4) << 24);              // M >> 4
 }
 __host__ __device__ constexpr uint32_t idesc_m128(int n, bool fp8) { return idesc_mn(128, n, fp8); }
 
