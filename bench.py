@@ -383,11 +383,13 @@ def report_ours(args, world, r) -> dict:
     # run back to back, and the clock record shows sw_power_cap under load)
     tc_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (2.0 if cfg.dtype == "fp8" else 1.0)
     t_roof_sus = max(t_hbm, acct["flops"] / (tc_sus * 1e12))
-    # router GEMM, top-k, refine, dispatch count, dispatch scan, gather, schedule, then the fused
-    # expert kernel (bf16 decode shape) or gate/up GEMM (+ W8A8 activation quantisation) and
-    # down GEMM, then combine
+    # router GEMM, selection (top-k + refined weights), dispatch count, dispatch scan, gather,
+    # schedule, then the fused expert kernel (bf16 decode shape) or gate/up GEMM (+ W8A8
+    # activation quantisation) and down GEMM, then combine
     fused = cfg.dtype == "bf16" and cfg.T * cfg.k <= 32 * cfg.E
-    launches = 9 if fused else (11 if cfg.dtype == "fp8" else 10)
+    launches = 8 if fused else (10 if cfg.dtype == "fp8" else 9)
+    if cfg.T >= 2048:  # selection and refinement as two launches
+        launches += 1
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

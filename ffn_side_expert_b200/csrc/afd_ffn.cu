@@ -31,7 +31,14 @@ namespace {
 // token stage.  Both keep two accumulator sets in TMEM so the epilogue of one unit overlaps the
 // next unit's MMAs.
 // tensor-core router: N tile of 64 tokens, three weight planes per stage
+// Router GEMM tiles: 64 tokens per unit for small micro-batches (more units to spread over the
+// SMs), 128 from kRouterWideT tokens up (an N = 128 MMA costs 64 cycles where an N = 64 one
+// still costs ~50, so the wide tile halves the issue time per token).  Both load the hidden
+// rows in 64-row boxes, so they share one tensor map.
 constexpr int kRouterBN = 64, kRouterStages = 3;
+constexpr int kRouterBNWide = 128, kRouterWideT = 1024;
+// Below this micro-batch size the top-k selection and the weight refinement run as one launch.
+constexpr int kSelectFusedMaxT = 2048;
 
 thread_local int g_create_cuda_error = 0;
 
@@ -333,6 +340,8 @@ cudaError_t set_all_gemm_attrs() {
   if (e != cudaSuccess) return e;
   e = set_gemm_attr<kRouterBN, kRouterStages, false, 2, false>();
   if (e != cudaSuccess) return e;
+  e = set_gemm_attr<kRouterBNWide, kRouterStages, false, 2, false>();
+  if (e != cudaSuccess) return e;
   e = set_pair_attrs<FP8, kWide>();
   if (e != cudaSuccess) return e;
   e = set_pair_attrs<FP8, kWideSingle>();
@@ -408,9 +417,9 @@ int pair_grid(int num_sms) {
 }
 
 // K split of the tensor-core router: enough units to cover the SMs, every split non-empty.
-void router_ksplit(int T, int H, int E, int sms, int* ksplit, int* kc_per) {
+void router_ksplit(int T, int H, int E, int sms, int bn, int* ksplit, int* kc_per) {
   const int kchunks = H / 64;
-  const int base = ((T + kRouterBN - 1) / kRouterBN) * ((E + 127) / 128);
+  const int base = ((T + bn - 1) / bn) * ((E + 127) / 128);
   const int want = std::max(1, std::min(kchunks, (sms + base - 1) / base));
   *kc_per = (kchunks + want - 1) / want;
   *ksplit = (kchunks + *kc_per - 1) / *kc_per;
@@ -429,13 +438,17 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
   CUtensorMap tm_h;
   if (!encode_2d(&tm_h, hidden, false, c.H, static_cast<uint64_t>(T), GemmShape<kRouterBN, false, 2>::kBoxRows))
     return AFD_ERR_INVALID_ARG;
+  static_assert(GemmShape<kRouterBN, false, 2>::kBoxRows == GemmShape<kRouterBNWide, false, 2>::kBoxRows,
+                "router tiles share the hidden-state map");
+  const bool wide = T >= kRouterWideT;
+  const int bn = wide ? kRouterBNWide : kRouterBN;
   int ksplit = 1, kc_per = 1;
-  router_ksplit(T, c.H, c.E, h->num_sms, &ksplit, &kc_per);
+  router_ksplit(T, c.H, c.E, h->num_sms, bn, &ksplit, &kc_per);
   GemmArgs a{};
   a.G = 1;
   a.single_rows = T;
   a.single_mt = (c.E + 127) / 128;
-  a.single_total = ((T + kRouterBN - 1) / kRouterBN) * a.single_mt * ksplit;
+  a.single_total = ((T + bn - 1) / bn) * a.single_mt * ksplit;
   a.kc_per = kc_per;
   a.K = c.H;
   a.a_rows = c.E;
@@ -445,12 +458,26 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
   a.out_ld = c.E;
   a.err = h->err;
   record(h, 0, s);
-  launch_gemm<kRouterBN, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
+  if (wide)
+    launch_gemm<kRouterBNWide, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
+  else
+    launch_gemm<kRouterBN, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
   record(h, 1, s);
   const float* bias = c.has_router_bias ? h->w.router_bias : nullptr;
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
-  router_refine_kernel<<<T, 32 * c.k, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, bias, c.H,
-                                             c.k, idx, w);
+  if (T < kSelectFusedMaxT) {
+    // small micro-batches: selection and refinement in one launch, up to four warps per selected
+    // expert splitting the dot product (few CTAs, so each one's chain of loads is the latency)
+    const int slices = std::max(1, std::min(4, 32 / c.k));
+    const int threads = std::max(256, 32 * c.k * slices);
+    router_select_kernel<<<T, threads, 0, s>>>(h->part, ksplit, bias, static_cast<const __nv_bfloat16*>(hidden),
+                                               h->w.router_w, T, c.E, c.H, c.k, idx, w);
+  } else {
+    // large ones: a warp per token selects, then a CTA per token refines (measured faster there
+    // than the one-launch form, whose warps wait on the selection)
+    router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
+    router_refine_kernel<<<T, 32 * c.k, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, bias,
+                                               c.H, c.k, idx, w);
+  }
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -693,7 +720,7 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   size_t part = 0;  // partial router logits [ksplit][T][E], largest over T <= T_max
   for (int T = 1; T <= c.T_max; ++T) {
     int ks, per;
-    router_ksplit(T, c.H, c.E, sms, &ks, &per);
+    router_ksplit(T, c.H, c.E, sms, T >= kRouterWideT ? kRouterBNWide : kRouterBN, &ks, &per);
     part = std::max(part, static_cast<size_t>(ks) * T * c.E);
   }
   h->part_floats = part;
