@@ -8,7 +8,7 @@ import torch
 
 import ffn_side_expert_b200 as afd
 import synth
-from layer_support import BF16_TOL, FP8_TOL, Layer, rel_max_err, to64
+from layer_support import BF16_TOL, FP8_TOL, W_TOL, Layer, rel_max_err, to64
 from oracle import moe
 
 pytestmark = pytest.mark.gpu
@@ -146,6 +146,24 @@ def test_wide_tiles_single_cta_when_i_is_not_a_multiple_of_256(dtype):
     L = Layer(cfg, redraws=_redraws(cfg))
     try:
         _check_layer(L, cfg.T, tol=FP8_TOL if dtype == "fp8" else BF16_TOL)
+    finally:
+        L.close()
+
+
+@pytest.mark.parametrize("T", [1500, 2100])
+def test_router_tiles_around_the_size_thresholds(T):
+    # T >= 1024: 128-token router GEMM tiles; T < 2048: selection and refinement in one launch,
+    # T >= 2048: separate selection and refinement kernels
+    cfg = synth.MoEConfig("thresholds", T=2100, H=256, E=16, k=4, I=256, S=1, seed=29)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        _check_layer(L, T)
+        idx, w = L.route(T)
+        _, ridx, rw = moe.route(L.hidden[:T], L.Wr, L.bias, cfg.k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        wg = w.cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(wg - rw)) <= W_TOL
+        assert np.max(np.abs(wg.sum(axis=1) - 1.0)) <= 1e-6
     finally:
         L.close()
 
