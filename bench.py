@@ -79,7 +79,7 @@ def algorithmic(cfg, counts) -> dict:
 def kernel_sources_sha256() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("gemm.cuh", "afd_ffn.cu"):
+    for name in ("gemm.cuh", "ptx.cuh", "common.cuh", "afd_ffn.cu"):
         with open(os.path.join(ROOT, "ffn_side_expert_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -87,7 +87,8 @@ def kernel_sources_sha256() -> str:
 
 def fused_traffic(cfg, acct):
     """Measured DRAM bytes per fused expert-kernel launch scaled to this workload's touched
-    experts, or None when the kernel sources changed since the capture."""
+    experts, or None when the kernel sources (the kernel, its PTX helpers and the file that
+    instantiates it) changed since the capture."""
     if kernel_sources_sha256() != MEASURED_TRAFFIC["sources_sha256"]:
         return None
     return int(round(MEASURED_TRAFFIC["bytes_per_touched_expert"] * acct["touched_experts"]))

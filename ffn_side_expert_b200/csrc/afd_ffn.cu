@@ -546,8 +546,9 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
     record(h, 7, s);
     return;
   }
-  if constexpr (!FP8 && !NARROW) {
-    if (h->act16 && !P::pair) {  // single-term down GEMM on f16 activations and the f16 copy of W2
+  if constexpr (!FP8 && !NARROW && !P::pair && P::bn1 == kAct16BN && P::bn2 == kAct16BN) {
+    // (the device schedule was built with P's N tiles, which the f16 kernels share)
+    if (h->act16) {  // single-term down GEMM on f16 activations and the f16 copy of W2
       GemmArgs a1 = g1;
       a1.mt_stride = 128;
       record(h, 5, s);
