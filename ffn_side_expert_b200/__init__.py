@@ -66,6 +66,11 @@ _SIGNATURES = {
     "afd_ffn_last_cuda_error": (ctypes.c_int, [_P]),
     "afd_ffn_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "afd_ffn_route_static": (ctypes.c_int, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "afd_ffn_dispatch_rows": (ctypes.c_int, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "afd_ffn_expert_rows": (ctypes.c_int, [_P, _P, _P, _I, _P, _P]),
+    "afd_ffn_copy_row_blocks": (ctypes.c_int, [_P, _P, _P, _I, _I, _P]),
+    "afd_ffn_combine_rows": (ctypes.c_int, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "afd_ffn_rows_error": (ctypes.c_int, []),
 }
 
 
@@ -198,6 +203,30 @@ def afd_ffn_route_static(hidden, router_w, router_bias, T, H, E, k, topk_idx, to
 
 
 AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS = 1 << 20
+
+
+# expert-parallel building blocks (declarations in include/afd_ffn.h)
+def afd_ffn_dispatch_rows(hidden, topk_idx, T, k, E, H, counts, offsets, pos, src, rows, scratch,
+                          stream=None) -> int:
+    return _lib.afd_ffn_dispatch_rows(_ptr(hidden), _ptr(topk_idx), T, k, E, H, _ptr(counts), _ptr(offsets),
+                                      _ptr(pos), _ptr(src), _ptr(rows), _ptr(scratch), _stream(stream))
+
+
+def afd_ffn_expert_rows(h, rows, counts, n_rows, Y, stream=None) -> int:
+    return _lib.afd_ffn_expert_rows(h, _ptr(rows), _ptr(counts), n_rows, _ptr(Y), _stream(stream))
+
+
+def afd_ffn_copy_row_blocks(src, dst, blocks, n_blocks, row_bytes, stream=None) -> int:
+    return _lib.afd_ffn_copy_row_blocks(_ptr(src), _ptr(dst), _ptr(blocks), n_blocks, row_bytes, _stream(stream))
+
+
+def afd_ffn_combine_rows(Y, Ys, topk_w, pos, T, k, H, out, stream=None) -> int:
+    return _lib.afd_ffn_combine_rows(_ptr(Y), _ptr(Ys), _ptr(topk_w), _ptr(pos), T, k, H, _ptr(out),
+                                     _stream(stream))
+
+
+def afd_ffn_rows_error() -> int:
+    return _lib.afd_ffn_rows_error()
 
 
 # ------------------------------------------------------------------ convenience wrapper

@@ -628,11 +628,11 @@ int run_combine(afd_ffn_handle* h, const float* w, const int32_t* pos, int T, vo
   const afd_ffn_cfg& c = h->cfg;
   record(h, 8, s);
   if (h->fp8)
-    combine_kernel<__nv_bfloat16><<<T, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->Y), w, pos, T, c.k,
+    combine_kernel<__nv_bfloat16><<<T, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->Y), nullptr, w, pos, T, c.k,
                                                     c.H, T * c.k, c.n_shared, static_cast<__nv_bfloat16*>(out),
                                                     h->err);
   else
-    combine_kernel<float><<<T, 256, 0, s>>>(h->Y, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
+    combine_kernel<float><<<T, 256, 0, s>>>(h->Y, nullptr, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
                                             static_cast<__nv_bfloat16*>(out), h->err);
   record(h, 9, s);
   AFD_CUDA(h, cudaGetLastError());
@@ -1055,4 +1055,124 @@ extern "C" int afd_ffn_route_static(const void* hidden, const float* router_w, c
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;
+}
+
+// ---------------------------------------------------------------------- expert parallelism
+// Building blocks of an expert-parallel layer whose exchange runs outside the library (the
+// dispatch/combine all-to-all of A/F 分离, section 机制): dispatch order and rows without a
+// handle, a handle's experts on rows that arrive already grouped by expert, row-block moves,
+// and the weighted combine of external expert outputs.  The allocation-free calls share one
+// file-scope device error word (indices outside [0, E) and positions out of range are skipped
+// and counted there; afd_ffn_rows_error reads and clears it).
+static __device__ int g_rows_err;
+
+namespace {
+std::mutex g_rows_err_mu;
+int* g_rows_err_dev[kMaxDevices] = {};
+
+int rows_err_word(int** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  if (dev < 0 || dev >= kMaxDevices) return AFD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_rows_err_mu);
+  if (!g_rows_err_dev[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_rows_err);
+    if (e != cudaSuccess) return cuda_fail(nullptr, e);
+    g_rows_err_dev[dev] = static_cast<int*>(p);
+  }
+  *out = g_rows_err_dev[dev];
+  return AFD_OK;
+}
+}  // namespace
+
+extern "C" int afd_ffn_dispatch_rows(const void* hidden, const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
+                                     int32_t H, int32_t* counts, int32_t* offsets, int32_t* pos, int32_t* src,
+                                     void* rows, int32_t* scratch, void* stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1 || E > kMaxExperts || k > E || H < 8 || H % 8 != 0) return AFD_ERR_INVALID_ARG;
+  if (!counts || !offsets || !scratch) return AFD_ERR_INVALID_ARG;
+  if (T > 0 && (!hidden || !topk_idx || !pos || !src || !rows || !aligned16(hidden) || !aligned16(rows)))
+    return AFD_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k > (1LL << 30)) return AFD_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  int st = rows_err_word(&err);
+  if (st != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nchunks = (T + kChunkTokens - 1) / kChunkTokens;
+  int32_t* chunk_counts = scratch;
+  int32_t* chunk_base = scratch + static_cast<size_t>(nchunks) * E;
+  if (T > 0)
+    dispatch_count_kernel<<<nchunks, kCountThreads, 0, s>>>(topk_idx, T, k, E, pos, chunk_counts, err);
+  dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(chunk_counts, nchunks, E, counts, offsets, chunk_base);
+  if (T > 0)
+    gather_rows_kernel<false><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), topk_idx, chunk_base, pos,
+                                                src, T, k, E, H, 0, static_cast<uint8_t*>(rows), nullptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_expert_rows(afd_ffn_handle* h, const void* rows, const int32_t* counts, int32_t n_rows,
+                                   float* Y, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  const afd_ffn_cfg& c = h->cfg;
+  if (c.k != 1 || c.n_shared != 0 || h->fp8) return AFD_ERR_UNSUPPORTED;
+  int st = check_T(h, n_rows);
+  if (st != AFD_OK) return st;
+  if (n_rows == 0) return AFD_OK;
+  if (!rows || !counts || !Y || !aligned16(rows) || !aligned16(Y)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  const size_t H = c.H;
+  AFD_CUDA(h, cudaMemcpyAsync(h->xp, rows, static_cast<size_t>(n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
+  // group offsets from the per-expert counts (one "chunk")
+  dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(counts, 1, c.E, h->counts, h->offsets, h->chunk_base);
+  AFD_CUDA(h, cudaGetLastError());
+  if ((st = run_expert_gemm(h, h->offsets, n_rows, s)) != AFD_OK) return st;
+  AFD_CUDA(h, cudaMemcpyAsync(Y, h->Y, static_cast<size_t>(n_rows) * H * 4, cudaMemcpyDeviceToDevice, s));
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_copy_row_blocks(const void* src, void* dst, const int32_t* blocks, int32_t n_blocks,
+                                       int32_t row_bytes, void* stream) {
+  if (n_blocks < 0 || row_bytes < 16 || row_bytes % 16 != 0) return AFD_ERR_INVALID_ARG;
+  if (n_blocks == 0) return AFD_OK;
+  if (!src || !dst || !blocks || !aligned16(src) || !aligned16(dst)) return AFD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  copy_row_blocks_kernel<<<dim3(static_cast<unsigned>(n_blocks), 16), 256, 0, s>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), blocks, row_bytes / 16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_combine_rows(const float* Y, const float* Ys, const float* topk_w, const int32_t* pos,
+                                    int32_t T, int32_t k, int32_t H, void* out, void* stream) {
+  if (T < 0 || k < 1 || k > 32 || H < 4 || H % 4 != 0) return AFD_ERR_INVALID_ARG;
+  if (T == 0) return AFD_OK;
+  if (!Y || !topk_w || !pos || !out || !aligned16(Y) || !aligned16(out) || (Ys && !aligned16(Ys)))
+    return AFD_ERR_INVALID_ARG;
+  int* err = nullptr;
+  int st = rows_err_word(&err);
+  if (st != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  combine_kernel<float><<<T, 256, 0, s>>>(Y, Ys, topk_w, pos, T, k, H, T * k, Ys ? 1 : 0,
+                                          static_cast<__nv_bfloat16*>(out), err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_rows_error(void) {
+  int* err = nullptr;
+  int st = rows_err_word(&err);
+  if (st != AFD_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  int word = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&word, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(err, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return word ? AFD_ERR_DEVICE_FLAG : AFD_OK;
 }

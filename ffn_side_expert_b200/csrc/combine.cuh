@@ -22,10 +22,12 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p, size_t i) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// Ys: the shared expert's rows [T][H], or nullptr when they follow the routed rows in Y.
 template <typename YT>
 __global__ void __launch_bounds__(256)
-combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int32_t* __restrict__ pos,
-               int T, int k, int H, int n_rows, int with_shared, __nv_bfloat16* __restrict__ out, int* err) {
+combine_kernel(const YT* __restrict__ Y, const YT* __restrict__ Ys, const float* __restrict__ w,
+               const int32_t* __restrict__ pos, int T, int k, int H, int n_rows, int with_shared,
+               __nv_bfloat16* __restrict__ out, int* err) {
   __shared__ int sp[32];
   __shared__ float sw[32];
   const int t = blockIdx.x;
@@ -36,7 +38,7 @@ combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int3
     sw[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
   }
   __syncthreads();
-  const YT* ys = Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
+  const YT* ys = Ys ? Ys + static_cast<size_t>(t) * H : Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
   for (int v = threadIdx.x; v < H / 4; v += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (sizeof(YT) == 4) {
@@ -83,6 +85,21 @@ combine_kernel(const YT* __restrict__ Y, const float* __restrict__ w, const int3
     packed.x = *reinterpret_cast<uint32_t*>(&lo);
     packed.y = *reinterpret_cast<uint32_t*>(&hi);
     reinterpret_cast<uint2*>(out + static_cast<size_t>(t) * H)[v] = packed;
+  }
+}
+
+// Copy blocks of rows: block b moves blocks[3b+2] rows of row_bytes from row blocks[3b] of src
+// to row blocks[3b+1] of dst.  blockIdx.x = block, blockIdx.y splits its rows; 16-byte moves.
+__global__ void __launch_bounds__(256)
+copy_row_blocks_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ blocks,
+                       int row_vecs) {
+  const int b = blockIdx.x;
+  const size_t s0 = static_cast<size_t>(blocks[3 * b]), d0 = static_cast<size_t>(blocks[3 * b + 1]);
+  const int rows = blocks[3 * b + 2];
+  for (int r = blockIdx.y; r < rows; r += gridDim.y) {
+    const uint4* sr = src + (s0 + r) * row_vecs;
+    uint4* dr = dst + (d0 + r) * row_vecs;
+    for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) dr[v] = sr[v];
   }
 }
 

@@ -1,0 +1,208 @@
+"""Expert parallelism for the FFN layer across the ranks of a torch.distributed group.
+
+Experts sit in contiguous blocks of E / world per rank; every rank holds a copy of the shared
+expert and routes its own micro-batch.  The exchange is the one the A/F split pages describe
+for the FFN side (A/F 分离 page, section 机制: each token's hidden state goes to the ranks that
+hold its experts, and their outputs come back for the weighted combine; the page's section
+通信账 counts those bytes).  Per forward:
+
+  1. route (fp32 router, top-k, renormalised softmax) and dispatch the rows in expert-major
+     order -- with experts in contiguous blocks that is also rank-major;
+  2. exchange the per-expert row counts, then the rows (all-to-all-v);
+  3. regroup the received rows from [source rank][local expert] to [local expert][source rank]
+     and run the local experts;
+  4. restore the received order and send the fp32 outputs back (all-to-all-v);
+  5. combine: out[t] = sum_j w[t,j] * Y[pos[t,j]] + shared(hidden[t]).
+
+Every arithmetic step runs in the library's kernels (ExpertParallelFfn's default backend);
+torch.distributed moves the bytes (NCCL between GPUs).  The backend is a parameter only so that
+the exchange can be exercised on CPU ranks.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+from . import (AFD_OK, AfdError, AfdFfn, afd_ffn_combine_rows, afd_ffn_copy_row_blocks, afd_ffn_dispatch_rows,
+               afd_ffn_expert_rows, afd_ffn_route_static)
+
+
+def block_tables(recv_counts: torch.Tensor):
+    """Row-block moves between the received order and the per-expert order.
+
+    recv_counts [world][E_local] (host int): rows that source rank s sent for local expert e,
+    received as blocks ordered (s, e).  Returns (to_grouped, to_received): int32 [n][3] tables
+    of (source row, destination row, rows) for moving (s, e) blocks into (e, s) order and back,
+    and the rows per local expert.
+    """
+    c = recv_counts.to(torch.int64)
+    world, el = c.shape
+    recv_off = torch.zeros_like(c)
+    flat = c.reshape(-1)
+    recv_off.view(-1)[1:] = torch.cumsum(flat, 0)[:-1]
+    per_expert = c.sum(0)
+    grp_off = torch.zeros_like(c)
+    expert_base = torch.zeros(el, dtype=torch.int64)
+    expert_base[1:] = torch.cumsum(per_expert, 0)[:-1]
+    for e in range(el):
+        run = int(expert_base[e])
+        for s in range(world):
+            grp_off[s, e] = run
+            run += int(c[s, e])
+    fwd, back = [], []
+    for s in range(world):
+        for e in range(el):
+            n = int(c[s, e])
+            if n:
+                fwd.append((int(recv_off[s, e]), int(grp_off[s, e]), n))
+                back.append((int(grp_off[s, e]), int(recv_off[s, e]), n))
+    as_t = (lambda rows: torch.tensor(rows, dtype=torch.int32).reshape(-1, 3))
+    return as_t(fwd), as_t(back), per_expert.to(torch.int32)
+
+
+@dataclass
+class WireBytes:
+    """Bytes one forward moved through the exchange on this rank."""
+    dispatch_sent: int      # rows sent for dispatch (to every rank, this one included) x row bytes
+    dispatch_remote: int    # ... of which to other ranks
+    combine_sent: int       # expert outputs sent back (fp32 rows)
+    combine_remote: int
+    tokens: int
+
+
+class CudaRowsBackend:
+    """The library's kernels for every step of the expert-parallel forward on one rank."""
+
+    def __init__(self, *, H, E, k, I, T_max, world, router_w, router_bias, local_w13, local_w2,
+                 shared_w13, shared_w2, device):
+        self.H, self.E, self.k, self.device = H, E, k, device
+        self.router_w, self.router_bias = router_w, router_bias
+        el = E // world
+        dummy_router = torch.zeros((el, H), dtype=torch.float32, device=device)  # unused by expert_rows
+        self.local = AfdFfn(T_max=world * T_max * k, H=H, E=el, k=1, I=I, n_shared=0, fp8=False,
+                            weights={"router_w": dummy_router, "w13": local_w13, "w2": local_w2})
+        self.shared = None
+        if shared_w13 is not None:
+            self.shared = AfdFfn(T_max=T_max, H=H, E=1, k=1, I=I, n_shared=0, fp8=False,
+                                 weights={"router_w": dummy_router[:1], "w13": shared_w13[None], "w2": shared_w2[None]})
+        self.scratch = torch.empty(2 * ((T_max + 127) // 128) * E, dtype=torch.int32, device=device)
+        self.keep = [dummy_router]
+
+    @staticmethod
+    def _ok(st, what):
+        if st != AFD_OK:
+            raise AfdError(st, what)
+
+    def route(self, hidden, T):
+        idx = torch.empty((T, self.k), dtype=torch.int32, device=self.device)
+        w = torch.empty((T, self.k), dtype=torch.float32, device=self.device)
+        self._ok(afd_ffn_route_static(hidden, self.router_w, self.router_bias, T, self.H, self.E, self.k, idx, w),
+                 "afd_ffn_route_static")
+        return idx, w
+
+    def dispatch(self, hidden, idx, T):
+        counts = torch.empty(self.E, dtype=torch.int32, device=self.device)
+        offsets = torch.empty(self.E + 1, dtype=torch.int32, device=self.device)
+        pos = torch.empty((T, self.k), dtype=torch.int32, device=self.device)
+        src = torch.empty(max(T * self.k, 1), dtype=torch.int32, device=self.device)
+        rows = torch.empty((max(T * self.k, 1), self.H), dtype=torch.bfloat16, device=self.device)
+        self._ok(afd_ffn_dispatch_rows(hidden, idx, T, self.k, self.E, self.H, counts, offsets, pos, src, rows,
+                                       self.scratch), "afd_ffn_dispatch_rows")
+        return counts, pos, rows
+
+    def copy_blocks(self, src, dst, blocks, row_bytes):
+        if blocks.shape[0]:
+            b = blocks.to(self.device)
+            self._ok(afd_ffn_copy_row_blocks(src, dst, b, b.shape[0], row_bytes), "afd_ffn_copy_row_blocks")
+
+    def experts(self, rows, per_expert, n):
+        Y = torch.empty((max(n, 1), self.H), dtype=torch.float32, device=self.device)
+        if n:
+            cnt = per_expert.to(self.device)
+            self._ok(afd_ffn_expert_rows(self.local.h, rows, cnt, n, Y), "afd_ffn_expert_rows")
+        return Y
+
+    def shared_expert(self, hidden, T):
+        if self.shared is None:
+            return None
+        Ys = torch.empty((max(T, 1), self.H), dtype=torch.float32, device=self.device)
+        cnt = torch.tensor([T], dtype=torch.int32, device=self.device)
+        self._ok(afd_ffn_expert_rows(self.shared.h, hidden, cnt, T, Ys), "afd_ffn_expert_rows (shared)")
+        return Ys
+
+    def combine(self, Y, Ys, w, pos, T):
+        out = torch.empty((max(T, 1), self.H), dtype=torch.bfloat16, device=self.device)
+        self._ok(afd_ffn_combine_rows(Y, Ys, w, pos, T, self.k, self.H, out), "afd_ffn_combine_rows")
+        return out[:T]
+
+    def close(self):
+        self.local.close()
+        if self.shared is not None:
+            self.shared.close()
+
+
+class ExpertParallelFfn:
+    """The MoE FFN layer with its routed experts split over the ranks of `group`.
+
+    Every rank calls forward() with its own micro-batch (the same T on all ranks is not
+    required).  `backend` defaults to CudaRowsBackend built from the arguments.
+    """
+
+    def __init__(self, *, H, E, k, I, T_max, router_w=None, router_bias=None, local_w13=None, local_w2=None,
+                 shared_w13=None, shared_w2=None, group=None, backend=None, device=None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if E % self.world:
+            raise ValueError("E must split evenly over the ranks")
+        self.H, self.E, self.k, self.el = H, E, k, E // self.world
+        self.device = device or (router_w.device if router_w is not None else None)
+        if backend is None and (router_w is None or local_w13 is None or local_w2 is None):
+            raise ValueError("router_w, local_w13 and local_w2 are required for the library backend")
+        self.backend = backend or CudaRowsBackend(
+            H=H, E=E, k=k, I=I, T_max=T_max, world=self.world, router_w=router_w, router_bias=router_bias,
+            local_w13=local_w13, local_w2=local_w2, shared_w13=shared_w13, shared_w2=shared_w2, device=self.device)
+        self.last_wire: WireBytes | None = None
+
+    def forward(self, hidden: torch.Tensor) -> torch.Tensor:
+        T, H, k = hidden.shape[0], self.H, self.k
+        b, g = self.backend, self.group
+        idx, w = b.route(hidden, T)
+        counts, pos, rows = b.dispatch(hidden, idx, T)
+        # 2. per-(rank, local expert) row counts, then the rows
+        send_c = counts.view(self.world, self.el).contiguous()
+        recv_c = torch.empty_like(send_c)
+        dist.all_to_all_single(recv_c, send_c, group=g)
+        send_c_h, recv_c_h = send_c.cpu(), recv_c.cpu()
+        send_split = send_c_h.sum(1).tolist()
+        recv_split = recv_c_h.sum(1).tolist()
+        n_send, n_recv = sum(send_split), sum(recv_split)
+        recv_rows = torch.empty((max(n_recv, 1), H), dtype=rows.dtype, device=rows.device)
+        dist.all_to_all_single(recv_rows[:n_recv], rows[:n_send], recv_split, send_split, group=g)
+        # 3. local experts on the rows regrouped by expert
+        to_grouped, to_received, per_expert = block_tables(recv_c_h)
+        grouped = torch.empty_like(recv_rows)
+        b.copy_blocks(recv_rows, grouped, to_grouped, H * rows.element_size())
+        Yg = b.experts(grouped, per_expert, n_recv)
+        # 4. outputs back in the order each source sent its rows
+        Yr = torch.empty_like(Yg)
+        b.copy_blocks(Yg, Yr, to_received, H * Yg.element_size())
+        Yback = torch.empty((max(n_send, 1), H), dtype=Yg.dtype, device=Yg.device)
+        dist.all_to_all_single(Yback[:n_send], Yr[:n_recv], send_split, recv_split, group=g)
+        # 5. weighted combine with the shared expert
+        Ys = b.shared_expert(hidden, T)
+        out = b.combine(Yback, Ys, w, pos, T)
+        rb, yb = H * rows.element_size(), H * Yg.element_size()
+        self.last_wire = WireBytes(
+            dispatch_sent=n_send * rb,
+            dispatch_remote=(n_send - send_split[self.rank]) * rb,
+            combine_sent=n_recv * yb,
+            combine_remote=(n_recv - recv_split[self.rank]) * yb,
+            tokens=T)
+        return out
+
+    def close(self):
+        if hasattr(self.backend, "close"):
+            self.backend.close()

@@ -195,6 +195,49 @@ int afd_ffn_route_static(const void *hidden, const float *router_w, const float 
                          int32_t T, int32_t H, int32_t E, int32_t k,
                          int32_t *topk_idx, float *topk_w, void *stream);
 
+/* ---- expert parallelism: building blocks ------------------------------------------
+ * An expert-parallel layer (experts split in contiguous blocks over ranks, hidden states sent
+ * to the experts' ranks and the outputs sent back: the dispatch / combine exchange of the A/F
+ * 分离 page, section 机制) runs its exchange outside the library; these calls do the rest.
+ * The allocation-free calls (no handle) share one device error word: expert indices outside
+ * [0, E) and positions outside the expert rows are skipped and flagged there. */
+
+/* Dispatch order and rows without a handle: for topk_idx [T][k] (device, global expert ids),
+ * writes counts [E], offsets [E+1] (exclusive prefix), pos [T][k] (dispatched row of each pair,
+ * -1 when skipped), src [T*k] (token of each row) and rows [T*k][H] bf16 = hidden rows in
+ * expert-major order, tokens ascending inside an expert -- so experts held in contiguous
+ * blocks per rank make the rows rank-major as well.  scratch: int32 [2 * ceil(T/128) * E]
+ * (device, caller-owned).  hidden, rows 16-byte aligned; H multiple of 8; 1 <= k <= min(E, 32),
+ * E <= 256.  Asynchronous on `stream`. */
+int afd_ffn_dispatch_rows(const void *hidden, const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
+                          int32_t H, int32_t *counts, int32_t *offsets, int32_t *pos, int32_t *src,
+                          void *rows, int32_t *scratch, void *stream);
+
+/* A handle's experts on rows that arrive grouped by expert: rows [n_rows][H] bf16 (device),
+ * counts [E] (device; rows of expert 0 first, then expert 1, ...; sum = n_rows) ->
+ * Y [n_rows][H] fp32, row r = the output of row r.  The handle must be bf16 with k == 1 and
+ * n_shared == 0 (a rank's expert block, or a replicated shared expert as E = 1);
+ * 0 <= n_rows <= T_max.  Asynchronous on `stream`. */
+int afd_ffn_expert_rows(afd_ffn_handle *h, const void *rows, const int32_t *counts, int32_t n_rows,
+                        float *Y, void *stream);
+
+/* Move blocks of rows: block b copies blocks[3b+2] rows of row_bytes bytes from row blocks[3b]
+ * of src to row blocks[3b+1] of dst (blocks: int32 [n_blocks][3], device).  Blocks must not
+ * overlap in dst.  row_bytes a multiple of 16; src, dst 16-byte aligned. */
+int afd_ffn_copy_row_blocks(const void *src, void *dst, const int32_t *blocks, int32_t n_blocks,
+                            int32_t row_bytes, void *stream);
+
+/* Weighted combine of external expert outputs: out[t] = sum_j topk_w[t][j] * Y[pos[t][j]]
+ * (+ Ys[t] when Ys != NULL), fp32 sum in j order with the shared row last, bf16 out [T][H].
+ * Y [T*k][H] fp32 in dispatch order, Ys [T][H] fp32 or NULL; pairs with pos < 0 are skipped.
+ * H multiple of 4; Y, Ys, out 16-byte aligned. */
+int afd_ffn_combine_rows(const float *Y, const float *Ys, const float *topk_w, const int32_t *pos,
+                         int32_t T, int32_t k, int32_t H, void *out, void *stream);
+
+/* Synchronise the device; AFD_ERR_DEVICE_FLAG if an allocation-free call skipped invalid data
+ * since the last check (the word is cleared), else AFD_OK. */
+int afd_ffn_rows_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,99 @@
+"""Expert parallelism over two gloo ranks on the CPU.
+
+The experts are split in contiguous blocks over the ranks; each rank routes its own
+micro-batch (of a different size), exchanges the per-expert row counts and the rows
+(all-to-all-v), runs its expert block and sends the outputs back for the combine.  The local
+compute here is the fp64 oracle (tests/ep_support.py), so what is checked is the exchange:
+every rank's output must equal the single-process oracle layer on its tokens, and the bytes
+on the wire must match the per-token account of the A/F split pages (dispatch rows: k per
+token; the combine returns the same rows).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from ffn_side_expert_b200.ep import ExpertParallelFfn, block_tables
+
+H, E, K, I = 16, 8, 2, 24
+TOKENS = {0: 12, 1: 9}
+
+
+def _weights():
+    rng = np.random.default_rng(7)
+    Wr = rng.normal(0, 1 / np.sqrt(H), (E, H))
+    experts = [(rng.normal(0, 1 / np.sqrt(H), (2 * I, H)), rng.normal(0, 1 / np.sqrt(I), (H, I)))
+               for _ in range(E + 1)]
+    return Wr, experts
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from ep_support import OracleRowsBackend
+        from oracle import moe
+        Wr, experts = _weights()
+        el = E // world
+        hidden = torch.from_numpy(np.random.default_rng(100 + rank).normal(0, 1, (TOKENS[rank], H)))
+        backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[rank * el:(rank + 1) * el],
+                                    shared=experts[E])
+        ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
+        out = ep.forward(hidden)
+        ref = moe.forward(hidden.numpy(), Wr, None, lambda e: {"w13": experts[e][0], "w2": experts[e][1]},
+                          E, K, 1)["out"]
+        q.put((rank, float(np.max(np.abs(out.numpy() - ref))), float(np.max(np.abs(ref))), ep.last_wire))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_match_the_single_process_layer():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29600 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, err, scale, wire in res:
+        assert err <= 1e-12 * max(scale, 1.0), (rank, err)
+        # every token sends k rows to the experts' ranks and gets k rows back
+        assert wire.tokens == TOKENS[rank]
+        assert wire.dispatch_sent == TOKENS[rank] * K * H * 8          # float64 rows in this test
+    sent = sum(w.dispatch_sent for _, _, _, w in res)
+    back = sum(w.combine_sent for _, _, _, w in res)
+    assert sent == back                                                # the same rows return
+
+
+def test_block_tables_regroup_and_restore():
+    # 3 source ranks x 2 local experts: rows arrive (source, expert)-major
+    c = torch.tensor([[2, 0], [1, 3], [0, 2]])
+    fwd, back, per_expert = block_tables(c)
+    assert per_expert.tolist() == [3, 5]
+    received = torch.arange(8)
+    grouped = torch.empty_like(received)
+    for s, d, n in fwd.tolist():
+        grouped[d:d + n] = received[s:s + n]
+    # expert 0: source 0's 2 rows (0,1), source 1's row (2); expert 1: source 1's 3 (3,4,5), source 2's 2 (6,7)
+    assert grouped.tolist() == [0, 1, 2, 3, 4, 5, 6, 7]      # (0,0) (1,0) | (1,1) (2,1)
+    restored = torch.empty_like(grouped)
+    for s, d, n in back.tolist():
+        restored[d:d + n] = grouped[s:s + n]
+    assert torch.equal(restored, received)
+
+
+def test_block_tables_interleave_sources_per_expert():
+    c = torch.tensor([[1, 1], [1, 1]])                 # 2 sources x 2 experts, one row each
+    fwd, _, per_expert = block_tables(c)
+    received = torch.tensor([10, 11, 20, 21])          # (s0,e0) (s0,e1) (s1,e0) (s1,e1)
+    grouped = torch.empty_like(received)
+    for s, d, n in fwd.tolist():
+        grouped[d:d + n] = received[s:s + n]
+    assert grouped.tolist() == [10, 20, 11, 21]        # expert 0 rows from both sources first
+    assert per_expert.tolist() == [2, 2]
