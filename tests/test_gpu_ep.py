@@ -31,7 +31,7 @@ def _redraws(cfg):
 def test_expert_parallel_layer_on_one_rank(T):
     cfg = synth.MoEConfig("ep", T=64, H=256, E=8, k=2, I=512, S=1, seed=30)
     L = Layer(cfg, redraws=_redraws(cfg))
-    port = 29700 + os.getpid() % 1000
+    port = 29700 + (os.getpid() + T) % 1000
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
     ep = None
     try:
