@@ -70,3 +70,21 @@ def test_null_handle_calls_fail_fast():
     assert afd.afd_ffn_get_error(None) == afd.AFD_ERR_INVALID_ARG
     assert afd.afd_ffn_set_stage_events(None, None) == afd.AFD_ERR_INVALID_ARG
     afd.afd_ffn_destroy(None)
+
+
+def test_expert_parallel_calls_fail_fast_on_bad_arguments():
+    # host-side checks only: none of these reaches the device
+    A = 4096  # a 16-byte aligned stand-in address
+    assert afd.afd_ffn_dispatch_rows(A, A, 4, 0, 8, 256, A, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG   # k = 0
+    assert afd.afd_ffn_dispatch_rows(A, A, 4, 9, 8, 256, A, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG   # k > E
+    assert afd.afd_ffn_dispatch_rows(A, A, 4, 2, 8, 12, A, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG    # H % 8
+    assert afd.afd_ffn_dispatch_rows(A, A, 4, 2, 8, 256, A, A, A, A, A + 2, A) == afd.AFD_ERR_INVALID_ARG  # rows
+    assert afd.afd_ffn_dispatch_rows(A, A, 4, 2, 8, 256, None, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG
+    assert afd.afd_ffn_expert_rows(None, A, A, 4, A) == afd.AFD_ERR_INVALID_ARG
+    assert afd.afd_ffn_copy_row_blocks(A, A, A, 1, 8) == afd.AFD_ERR_INVALID_ARG                        # 8-byte rows
+    assert afd.afd_ffn_copy_row_blocks(A, A, A, -1, 16) == afd.AFD_ERR_INVALID_ARG
+    assert afd.afd_ffn_copy_row_blocks(A, A, A, 0, 16) == afd.AFD_OK                                    # nothing to do
+    assert afd.afd_ffn_combine_rows(A, None, A, A, 4, 33, 256, A) == afd.AFD_ERR_INVALID_ARG            # k > 32
+    assert afd.afd_ffn_combine_rows(A, None, A, A, 4, 2, 6, A) == afd.AFD_ERR_INVALID_ARG               # H % 4
+    assert afd.afd_ffn_combine_rows(A, A + 4, A, A, 4, 2, 256, A) == afd.AFD_ERR_INVALID_ARG            # Ys align
+    assert afd.afd_ffn_combine_rows(A, None, A, A, 0, 2, 256, A) == afd.AFD_OK                          # T = 0
