@@ -36,13 +36,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
 # of the decode shape, from a one-pass ncu capture of two launches at T=256, H=7168, E=256,
-# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 128 245 504 and
-# 23 142 697 984 bytes for 257 touched experts.  Traffic grows with the experts whose weights
+# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 076 790 784 and
+# 23 081 380 864 bytes for 257 touched experts.  Traffic grows with the experts whose weights
 # are streamed, and it is reported only while the kernel source and its instantiation are the
 # ones that were captured.
 MEASURED_TRAFFIC = {
-    "sources_sha256": "3baa67f270f746cbbc7efbd78c1a8841474bf53d082c083d257ba422051725b7",
-    "bytes_per_touched_expert": (23128245504 + 23142697984) / 2 / 257,
+    "sources_sha256": "4ce71176ccf4a25e5657cece790d582a933f0b7741fba5a16a1d09785e611c1c",
+    "bytes_per_touched_expert": (23076790784 + 23081380864) / 2 / 257,
 }
 METRIC = "MoE-FFN tokens/s/layer"
 
