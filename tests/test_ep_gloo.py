@@ -43,9 +43,12 @@ def _worker(rank, world, port, q):
                                     shared=experts[E])
         ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
         out = ep.forward(hidden)
+        from oracle import comm
+        idx = moe.route(hidden.numpy(), Wr, None, K)[1]
+        account = comm.element_bytes(idx, H, 8)          # the oracle's per-direction account
         ref = moe.forward(hidden.numpy(), Wr, None, lambda e: {"w13": experts[e][0], "w2": experts[e][1]},
                           E, K, 1)["out"]
-        q.put((rank, float(np.max(np.abs(out.numpy() - ref))), float(np.max(np.abs(ref))), ep.last_wire))
+        q.put((rank, float(np.max(np.abs(out.numpy() - ref))), float(np.max(np.abs(ref))), ep.last_wire, account))
     finally:
         dist.destroy_process_group()
 
@@ -61,13 +64,14 @@ def test_two_ranks_match_the_single_process_layer():
         p.join(180)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(2))
-    for rank, err, scale, wire in res:
+    for rank, err, scale, wire, account in res:
         assert err <= 1e-12 * max(scale, 1.0), (rank, err)
         # every token sends k rows to the experts' ranks and gets k rows back
         assert wire.tokens == TOKENS[rank]
         assert wire.dispatch_sent == TOKENS[rank] * K * H * 8          # float64 rows in this test
-    sent = sum(w.dispatch_sent for _, _, _, w in res)
-    back = sum(w.combine_sent for _, _, _, w in res)
+        assert wire.dispatch_sent == account                           # = the oracle's element account
+    sent = sum(r[3].dispatch_sent for r in res)
+    back = sum(r[3].combine_sent for r in res)
     assert sent == back                                                # the same rows return
 
 
