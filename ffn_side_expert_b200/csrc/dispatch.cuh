@@ -198,8 +198,10 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __re
 }
 
 // W8A8: quantise each row of the fp32 SwiGLU output act32 [R][I] to e4m3 with its own scale,
-// the same rule as the hidden rows.  One warp per row, eight rows per CTA; the second pass over
-// a row reads it from L1.
+// the same rule as the hidden rows.  One warp per row, eight rows per CTA.  Rows of up to
+// kActRegVecs x 128 values stay in registers between the amax and the quantisation (one pass
+// over memory); longer rows read their second pass back through the cache.
+constexpr int kActRegVecs = 16;  // float4 per lane: I <= 2048
 __global__ void __launch_bounds__(256)
 quantize_act_kernel(const float* __restrict__ act32, int R, int I, uint8_t* __restrict__ actq,
                     float* __restrict__ ascale) {
@@ -207,24 +209,40 @@ quantize_act_kernel(const float* __restrict__ act32, int R, int I, uint8_t* __re
   const size_t r = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (r >= static_cast<size_t>(R)) return;
   const float4* row = reinterpret_cast<const float4*>(act32 + r * I);
-  float amax = 0.f;
-  for (int v = lane; v < I / 4; v += 32) {
-    const float4 x = row[v];
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
-  }
-  amax = warp_max(amax);
-  const float scale = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
   uint32_t* out = reinterpret_cast<uint32_t*>(actq + r * I);
-  for (int v = lane; v < I / 4; v += 32) {
-    const float4 x = row[v];
+  const int nv = I / 128;  // float4 per lane
+  auto quant4 = [](const float4 x, float scale) {
     const float xv[4] = {x.x, x.y, x.z, x.w};
     uint32_t packed = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(xv[i], scale), __NV_SATFINITE, __NV_E4M3))
                 << (8 * i);
-    out[v] = packed;
+    return packed;
+  };
+  auto amax4 = [](const float4 x) { return fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))); };
+  float amax = 0.f;
+  if (nv <= kActRegVecs) {
+    float4 x[kActRegVecs];
+#pragma unroll
+    for (int i = 0; i < kActRegVecs; ++i) {
+      if (i < nv) {
+        x[i] = row[lane + 32 * i];
+        amax = fmaxf(amax, amax4(x[i]));
+      }
+    }
+    amax = warp_max(amax);
+    const float scale = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
+#pragma unroll
+    for (int i = 0; i < kActRegVecs; ++i)
+      if (i < nv) out[lane + 32 * i] = quant4(x[i], scale);
+    if (lane == 0) ascale[r] = scale;
+    return;
   }
+  for (int v = lane; v < I / 4; v += 32) amax = fmaxf(amax, amax4(row[v]));
+  amax = warp_max(amax);
+  const float scale = amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.0f;
+  for (int v = lane; v < I / 4; v += 32) out[v] = quant4(row[v], scale);
   if (lane == 0) ascale[r] = scale;
 }
 
