@@ -30,7 +30,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "MoEConfig", "CONFIGS", "get_config", "rng_for",
+    "MoEConfig", "CONFIGS", "get_config", "rng_for", "gen_experts_on",
     "gen_hidden", "redraw_row", "gen_router", "gen_expert", "gen_experts",
     "load_redraws", "REDRAW_TABLE",
 ]
@@ -182,6 +182,33 @@ def gen_expert(cfg: MoEConfig, e: int) -> dict:
         return {"w13": q13, "w2": q2, "w13_scale": s13, "w2_scale": s2}
     return {"w13": torch.from_numpy(w13).to(torch.bfloat16),
             "w2": torch.from_numpy(w2).to(torch.bfloat16)}
+
+
+def gen_experts_on(cfg: MoEConfig, device, threads: int | None = None) -> dict:
+    """The same stacked experts as gen_experts, written expert by expert into tensors on
+    ``device``; the host holds only the experts in flight (a few hundred MB), not the stack."""
+    n = cfg.E + cfg.S
+    wdt = torch.float8_e4m3fn if cfg.dtype == "fp8" else torch.bfloat16
+    out = {"w13": torch.empty((n, 2 * cfg.I, cfg.H), dtype=wdt, device=device),
+           "w2": torch.empty((n, cfg.H, cfg.I), dtype=wdt, device=device)}
+    if cfg.dtype == "fp8":
+        out["w13_scale"] = torch.empty((n, 2 * cfg.I), dtype=torch.float32, device=device)
+        out["w2_scale"] = torch.empty((n, cfg.H), dtype=torch.float32, device=device)
+
+    def fill(e):
+        d = gen_expert(cfg, e)
+        for key, v in d.items():
+            out[key][e].copy_(v)
+
+    threads = threads or max(1, min(8, len(os.sched_getaffinity(0))))
+    torch_threads = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(fill, range(n)))
+    finally:
+        torch.set_num_threads(torch_threads)
+    return out
 
 
 def gen_experts(cfg: MoEConfig, threads: int | None = None, pin: bool = False) -> dict:
