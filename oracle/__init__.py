@@ -12,7 +12,7 @@ Modules
 
 Pins (every function is checked against something other than itself, in tests marked
 ``not gpu``): closed forms of silu; a hand-derived worked example of one SwiGLU expert
-(tests/golden/swiglu_worked_example.json); the E=1, k=1 layer against a dense FFN; top-k
+(tests/test_oracle_expert.py::test_swiglu_worked_example); the E=1, k=1 layer against a dense FFN; top-k
 against a brute-force search over all k-subsets; the two gate-weight formulas against each
 other and sum-to-one; the dispatch order against an O(T^2 k) recount; the combine against
 a one-hot gather and linearity; every e4m3 code against a printed table and against
