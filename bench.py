@@ -16,6 +16,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -43,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # are streamed, and it is reported only while the kernel source and its instantiation are the
 # ones that were captured.
 MEASURED_TRAFFIC = {
-    "sources_sha256": "4ce71176ccf4a25e5657cece790d582a933f0b7741fba5a16a1d09785e611c1c",
+    "sources_sha256": "e79c1ebd330be23c2d966e0fbbce8a6fbf48fd621f8c83d326de1e01e904dd79",
     "bytes_per_touched_expert": (23076790784 + 23081380864) / 2 / 257,
 }
 METRIC = "MoE-FFN tokens/s/layer"
@@ -483,6 +484,142 @@ def run_reference(args, rank, world):
     }
 
 
+# ----------------------------------------------------------------------------- micro-pipeline period
+def _busy_until(t_end_ns: int) -> None:
+    while time.monotonic_ns() < t_end_ns:
+        pass
+
+
+def pipeline_period(layer, hidden_host, T, t_a_ms, n_slots, rounds, ref_out=None):
+    """One attention stub and the FFN serving loop, `n_slots` micro-batches in flight.
+
+    The attention side is a host stub: per micro-batch it writes the seeded hidden rows into a
+    mailbox slot (one memmove on its own thread) and holds the thread busy until t_a has passed
+    since it started, then posts the slot; it waits for a slot's output before it starts that
+    slot's next micro-batch.  The
+    FFN side is the library's serving loop (H2D, afd_ffn_forward, D2H on three streams).  The
+    period is the mean interval between outputs landing in host memory (the times the
+    library stamps when each D2H completes), after the first round.  Returns (period_ms,
+    outputs that differ from ref_out, service stats, median post->take and take->landed ms)."""
+    from ffn_side_expert_b200.service import FfnService, Mailbox
+    mb = Mailbox(n_slots, T, hidden_host.shape[1])
+    svc = FfnService(layer, mb)
+    t_a_ns = int(t_a_ms * 1e6)
+    rows = hidden_host[:T].contiguous()
+
+    def attention(slot):
+        t_end = time.monotonic_ns() + t_a_ns
+        mb.write_input(slot, rows)
+        _busy_until(t_end)
+
+    nbytes = T * hidden_host.shape[1] * 2
+    ref_bytes = None if ref_out is None else ref_out[:T].contiguous().view(torch.int16).numpy().tobytes()
+    landed, pickup, serve, tl, mismatches = [], [], [], [], 0
+    try:
+        for s in range(n_slots):
+            attention(s)
+            mb.post(s, T)
+        for r in range(rounds):
+            for s in range(n_slots):
+                mb.wait(s, timeout_s=60.0)
+                t_post, t_take, t_done = mb.times_ns(s)
+                landed.append(t_done)
+                if r:
+                    pickup.append((t_take - t_post) / 1e6)
+                    serve.append((t_done - t_take) / 1e6)
+                    tl.append(svc.timeline(s))
+                if ref_bytes is not None and r in (0, rounds - 1):   # single-threaded byte compare
+                    mismatches += int(ctypes.string_at(mb.output(s).data_ptr(), nbytes) != ref_bytes)
+                if r < rounds - 1:
+                    attention(s)
+                    mb.post(s, T)
+    finally:
+        stats = svc.stop()
+        mb.close()
+    w = n_slots
+    period_mean = (landed[-1] - landed[w]) / (len(landed) - 1 - w) / 1e6
+    # per-round periods (n_slots outputs each) after the first round; the median is robust to a
+    # host stall in one round, the mean is reported beside it
+    rounds_ms = [(landed[i + n_slots] - landed[i]) / n_slots / 1e6 for i in range(w, len(landed) - n_slots)]
+    period = statistics.median(rounds_ms)
+    # device timeline: layer start / end of each micro-batch on one clock (the service's origin)
+    spans = sorted((m[0] + m[2], m[0] + m[3]) for m in tl)
+    gaps = [b0 - a1 for (_, a1), (b0, _) in zip(spans, spans[1:])]
+    med = lambda xs: round(statistics.median(xs), 4)  # noqa: E731
+    parts = {"post_to_take_ms": med(pickup), "take_to_landed_ms": med(serve),
+             "period_mean_ms": round(period_mean, 4),
+             "h2d_ms": med([m[1] for m in tl]), "h2d_end_to_layer_ms": med([m[2] - m[1] for m in tl]),
+             "layer_ms": med([m[3] - m[2] for m in tl]),
+             "layer_gap_ms": med(gaps) if gaps else None,
+             "d2h_after_layer_ms": med([m[4] - m[3] for m in tl]),
+             # host take -> landed minus the device span H2D start -> D2H end: enqueue latency
+             # plus the time from the D2H end to the completion reaching the mailbox
+             "host_overhead_ms": med([sv - m[4] for sv, m in zip(serve, tl)])}
+    return period, mismatches, stats, parts
+
+
+def run_period(args) -> dict:
+    """The micro-pipeline period of the A/F split (A/F 分离 page, section 深入推导, 微流水): the
+    steady-state period with the attention of one micro-batch overlapping the FFN of another,
+    against max(t_a, t_f) + t_comm and against t_a + t_f when both share one device."""
+    import ffn_side_expert_b200 as afd
+    cfg = workload(args)
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    hidden, Wr, bias, dev = build_inputs(cfg, device)
+    layer = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S,
+                       fp8=cfg.dtype == "fp8", weights=dev)
+    T, H = cfg.T, cfg.H
+    h = hidden.to(device)
+    out = torch.empty_like(h)
+    for _ in range(args.warmup):
+        layer.forward(h, out)
+    torch.cuda.synchronize()
+    ref_out = out.cpu()
+    if layer.get_error() != afd.AFD_OK:
+        raise RuntimeError("device error word set during warm-up")
+
+    def device_ms(fn, reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    reps = max(args.steps, 5)
+    t_f = device_ms(lambda: layer.forward(h, out), reps)
+    host_in = hidden.pin_memory()
+    host_out = torch.empty_like(host_in).pin_memory()
+    t_h2d = device_ms(lambda: h.copy_(host_in, non_blocking=True), reps)
+    t_d2h = device_ms(lambda: host_out.copy_(out, non_blocking=True), reps)
+    t_comm = t_h2d + t_d2h
+    points, bad = [], 0
+    rounds = max(args.steps, 8)
+    for ratio in (0.5, 1.0, 1.5):
+        t_a = ratio * t_f
+        for slots in (1, 2):
+            period, mism, st, parts = pipeline_period(layer, host_in, T, t_a, slots, rounds, ref_out)
+            bad += mism
+            if st.status != afd.AFD_OK or st.device_status != afd.AFD_OK:
+                raise afd.AfdError(st.status or st.device_status, "FFN service")
+            model = (max(t_a, t_f) if slots > 1 else t_a + t_f) + t_comm
+            points.append({"t_a_ms": round(t_a, 4), "slots": slots, "period_ms": round(period, 4),
+                           "model_ms": round(model, 4), "colocated_ms": round(t_a + t_f, 4),
+                           "period_over_colocated": round(period / (t_a + t_f), 3), **parts})
+    return {
+        "metric": "FFN-service micro-pipeline period", "unit": "ms", "higher_is_better": False,
+        "config": {"workload": workload_label(args), "T": T, "H": H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+                   "n_shared": cfg.S, "weights": cfg.dtype, "attention": "host stub, busy t_a per micro-batch",
+                   "link": "PCIe host<->device copies (pinned)", "rounds": rounds},
+        "t_f_ms": round(t_f, 4), "t_comm_ms": {"h2d": round(t_h2d, 4), "d2h": round(t_d2h, 4), "sum": round(t_comm, 4)},
+        "models": {"slots=1": "t_a + t_f + t_comm", "slots=2": "max(t_a, t_f) + t_comm", "colocated": "t_a + t_f"},
+        "points": points, "outputs_bit_equal_to_forward": bad == 0,
+    }
+
+
 # ----------------------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -497,6 +634,8 @@ def main(argv=None):
                     help="profiling only: override the micro-batch size (a smaller case of the same kernels)")
     ap.add_argument("--E", type=int, default=None,
                     help="profiling only: override the number of routed experts")
+    ap.add_argument("--period", action="store_true",
+                    help="measure the FFN-service micro-pipeline period with a host attention stub (1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -504,6 +643,12 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.period:
+        if world > 1:
+            ap.error("--period runs on one GPU")
+        print(json.dumps(run_period(args)), flush=True)
+        return 0
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)

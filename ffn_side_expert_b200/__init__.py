@@ -27,6 +27,9 @@ AFD_ERR_CUDA = -4
 AFD_ERR_DEVICE_FLAG = -5
 AFD_ERR_DEVICE_TIMEOUT = -6
 AFD_ERR_NO_DEVICE = -7
+AFD_ERR_TIMEOUT = -8
+AFD_ERR_STOPPED = -9
+AFD_MAILBOX_PINNED = 1
 AFD_DT_BF16 = 0
 AFD_DT_FP8_E4M3 = 1
 AFD_FFN_NUM_STAGES = 9
@@ -47,8 +50,14 @@ class afd_ffn_weights(ctypes.Structure):
                 ("w13_scale", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p)]
 
 
+class afd_ffn_service_stats(ctypes.Structure):
+    _fields_ = [("served", ctypes.c_int64), ("status", ctypes.c_int32), ("device_status", ctypes.c_int32),
+                ("last_cuda_error", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
+_L = ctypes.c_int64
 _SIGNATURES = {
     "afd_ffn_create": (ctypes.c_int, [ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(afd_ffn_weights),
                                       ctypes.POINTER(ctypes.c_void_p)]),
@@ -71,6 +80,19 @@ _SIGNATURES = {
     "afd_ffn_copy_row_blocks": (ctypes.c_int, [_P, _P, _P, _I, _I, _P]),
     "afd_ffn_combine_rows": (ctypes.c_int, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "afd_ffn_rows_error": (ctypes.c_int, []),
+    "afd_ffn_get_info": (ctypes.c_int, [_P, ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(ctypes.c_int32)]),
+    "afd_ffn_mailbox_create": (ctypes.c_int, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_void_p)]),
+    "afd_ffn_mailbox_destroy": (None, [_P]),
+    "afd_ffn_mailbox_input": (_P, [_P, _I]),
+    "afd_ffn_mailbox_output": (_P, [_P, _I]),
+    "afd_ffn_mailbox_post": (ctypes.c_int, [_P, _I, _I]),
+    "afd_ffn_mailbox_wait": (ctypes.c_int, [_P, _I, _L]),
+    "afd_ffn_mailbox_take": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), _L]),
+    "afd_ffn_mailbox_complete": (ctypes.c_int, [_P, _I, _I]),
+    "afd_ffn_mailbox_times": (ctypes.c_int, [_P, _I, ctypes.POINTER(ctypes.c_int64)]),
+    "afd_ffn_service_start": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(ctypes.c_void_p)]),
+    "afd_ffn_service_stop": (ctypes.c_int, [_P, ctypes.POINTER(afd_ffn_service_stats)]),
+    "afd_ffn_service_slot_timeline": (ctypes.c_int, [_P, _I, ctypes.POINTER(ctypes.c_float)]),
 }
 
 
@@ -227,6 +249,81 @@ def afd_ffn_combine_rows(Y, Ys, topk_w, pos, T, k, H, out, stream=None) -> int:
 
 def afd_ffn_rows_error() -> int:
     return _lib.afd_ffn_rows_error()
+
+
+def afd_ffn_get_info(h):
+    """Returns (status, afd_ffn_cfg, device)."""
+    cfg, dev = afd_ffn_cfg(), ctypes.c_int32(-1)
+    st = _lib.afd_ffn_get_info(h, ctypes.byref(cfg), ctypes.byref(dev))
+    return st, cfg, dev.value
+
+
+# FFN service: mailbox and serving loop (declarations in include/afd_ffn.h)
+def afd_ffn_mailbox_create(n_slots, T_max, H, flags=0):
+    """Returns (status, mailbox or None)."""
+    mb = ctypes.c_void_p()
+    st = _lib.afd_ffn_mailbox_create(n_slots, T_max, H, flags, ctypes.byref(mb))
+    return st, (mb.value if st == AFD_OK else None)
+
+
+def afd_ffn_mailbox_destroy(mb) -> None:
+    _lib.afd_ffn_mailbox_destroy(mb)
+
+
+def afd_ffn_mailbox_input(mb, slot):
+    return _lib.afd_ffn_mailbox_input(mb, slot)
+
+
+def afd_ffn_mailbox_output(mb, slot):
+    return _lib.afd_ffn_mailbox_output(mb, slot)
+
+
+def afd_ffn_mailbox_post(mb, slot, T) -> int:
+    return _lib.afd_ffn_mailbox_post(mb, slot, T)
+
+
+def afd_ffn_mailbox_wait(mb, slot, timeout_us) -> int:
+    return _lib.afd_ffn_mailbox_wait(mb, slot, timeout_us)
+
+
+def afd_ffn_mailbox_take(mb, timeout_us):
+    """Returns (status, slot, T)."""
+    slot, T = ctypes.c_int32(-1), ctypes.c_int32(-1)
+    st = _lib.afd_ffn_mailbox_take(mb, ctypes.byref(slot), ctypes.byref(T), timeout_us)
+    return st, slot.value, T.value
+
+
+def afd_ffn_mailbox_complete(mb, slot, status) -> int:
+    return _lib.afd_ffn_mailbox_complete(mb, slot, status)
+
+
+def afd_ffn_mailbox_times(mb, slot):
+    """Returns (status, (post_ns, take_ns, done_ns))."""
+    t = (ctypes.c_int64 * 3)()
+    st = _lib.afd_ffn_mailbox_times(mb, slot, t)
+    return st, tuple(t)
+
+
+def afd_ffn_service_start(h, mb, stream=None):
+    """Returns (status, service or None)."""
+    svc = ctypes.c_void_p()
+    st = _lib.afd_ffn_service_start(h, mb, _stream(stream), ctypes.byref(svc))
+    return st, (svc.value if st == AFD_OK else None)
+
+
+def afd_ffn_service_slot_timeline(svc, slot):
+    """Returns (status, (origin->H2D start, H2D end, layer start, layer end, D2H end)) in ms,
+    the last four from the H2D start."""
+    ms = (ctypes.c_float * 5)()
+    st = _lib.afd_ffn_service_slot_timeline(svc, slot, ms)
+    return st, tuple(ms)
+
+
+def afd_ffn_service_stop(svc):
+    """Returns (status, afd_ffn_service_stats)."""
+    stats = afd_ffn_service_stats()
+    st = _lib.afd_ffn_service_stop(svc, ctypes.byref(stats))
+    return st, stats
 
 
 # ------------------------------------------------------------------ convenience wrapper

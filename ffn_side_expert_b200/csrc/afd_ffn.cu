@@ -682,11 +682,20 @@ const char* afd_ffn_strerror(int status) {
     case AFD_ERR_DEVICE_FLAG: return "device skipped invalid data (expert index or position)";
     case AFD_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case AFD_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+    case AFD_ERR_TIMEOUT: return "a bounded host wait timed out";
+    case AFD_ERR_STOPPED: return "the FFN service stopped before serving the slot";
     default: return "unknown status";
   }
 }
 
 int afd_ffn_last_cuda_error(const afd_ffn_handle* h) { return h ? h->last_cuda_error : g_create_cuda_error; }
+
+int afd_ffn_get_info(const afd_ffn_handle* h, afd_ffn_cfg* cfg, int32_t* device) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  if (cfg) *cfg = h->cfg;
+  if (device) *device = h->device;
+  return AFD_OK;
+}
 
 int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_ffn_handle** out) {
   if (!out) return AFD_ERR_INVALID_ARG;

@@ -54,6 +54,8 @@ extern "C" {
 #define AFD_ERR_DEVICE_FLAG    (-5)  /* afd_ffn_get_error: kernels skipped invalid data        */
 #define AFD_ERR_DEVICE_TIMEOUT (-6)  /* afd_ffn_get_error: a bounded on-device wait gave up    */
 #define AFD_ERR_NO_DEVICE      (-7)  /* no sm_100 device current                               */
+#define AFD_ERR_TIMEOUT        (-8)  /* a bounded host-side wait gave up                        */
+#define AFD_ERR_STOPPED        (-9)  /* the FFN service stopped before it served the slot       */
 
 /* ---- configuration ---------------------------------------------------------------- */
 typedef enum { AFD_DT_BF16 = 0, AFD_DT_FP8_E4M3 = 1 } afd_dtype;
@@ -237,6 +239,83 @@ int afd_ffn_combine_rows(const float *Y, const float *Ys, const float *topk_w, c
 /* Synchronise the device; AFD_ERR_DEVICE_FLAG if an allocation-free call skipped invalid data
  * since the last check (the word is cleared), else AFD_OK. */
 int afd_ffn_rows_error(void);
+
+/* The configuration and device of a handle (host only; either output may be NULL). */
+int afd_ffn_get_info(const afd_ffn_handle *h, afd_ffn_cfg *cfg, int32_t *device);
+
+/* ---- FFN service: mailbox and serving loop ----------------------------------------
+ * The FFN side of an A/F split runs a loop per layer: take the activations the attention side
+ * sent, run the layer, send the output back (vLLM AFD Plugin page, section 系統架構, "2. FFN
+ * Service").  With several micro-batches in flight the attention of one overlaps the FFN of
+ * another, so the steady-state period is max(t_a, t_f) + t_comm instead of t_a + t_f when both
+ * share a device (A/F 分离 page, section 深入推导, 微流水).
+ *
+ * The mailbox is the connector between the two sides on one host: n_slots slots, each an input
+ * buffer [T_max][H] bf16 (the hidden states of one micro-batch) and an output buffer of the
+ * same shape (the layer's output), both HOST memory owned by the mailbox.  A slot moves
+ *     free --post--> posted --take--> taken --complete--> done | failed --post--> ...
+ * The producer (attention side) writes the input, posts, later waits and reads the output; the
+ * consumer (one thread: the service, or a caller's loop) takes slots in post order and
+ * completes them.  Producers on several threads may post distinct slots.  Waits are bounded:
+ * they spin for about 20 us, then sleep until the state changes or the time is up; a wait that
+ * gives up returns AFD_ERR_TIMEOUT and leaves the slot as it was.  Times are CLOCK_MONOTONIC
+ * nanoseconds. */
+typedef struct afd_ffn_mailbox afd_ffn_mailbox;
+typedef struct afd_ffn_service afd_ffn_service;
+
+#define AFD_MAILBOX_PINNED 1   /* flags: buffers in page-locked memory (needs a CUDA device) */
+
+/* n_slots >= 1, T_max >= 1, H >= 8 and a multiple of 8.  Buffers are 64-byte aligned and
+ * zero-filled.  Without AFD_MAILBOX_PINNED they are ordinary host memory (no device needed).
+ * AFD_ERR_CUDA when the page-locked allocation fails. */
+int afd_ffn_mailbox_create(int32_t n_slots, int32_t T_max, int32_t H, int32_t flags,
+                           afd_ffn_mailbox **out);
+/* No consumer may run on the mailbox (stop the service first).  NULL is a no-op. */
+void afd_ffn_mailbox_destroy(afd_ffn_mailbox *mb);
+/* Host pointer of a slot's input / output buffer; NULL for a bad slot. */
+void *afd_ffn_mailbox_input(afd_ffn_mailbox *mb, int32_t slot);
+void *afd_ffn_mailbox_output(afd_ffn_mailbox *mb, int32_t slot);
+
+/* Producer: hand over the first T rows of the slot's input (0 <= T <= T_max).  The slot must
+ * be free, done or failed, else AFD_ERR_INVALID_ARG. */
+int afd_ffn_mailbox_post(afd_ffn_mailbox *mb, int32_t slot, int32_t T);
+/* Producer: wait up to timeout_us for the posted slot to finish.  AFD_OK once done (the first
+ * T rows of the output are valid), the consumer's status once failed (AFD_ERR_STOPPED when the
+ * service stopped first), AFD_ERR_TIMEOUT, or AFD_ERR_INVALID_ARG for a slot never posted. */
+int afd_ffn_mailbox_wait(afd_ffn_mailbox *mb, int32_t slot, int64_t timeout_us);
+
+/* Consumer (one thread at a time): the oldest posted slot and its T, waiting up to timeout_us;
+ * AFD_ERR_TIMEOUT when none was posted in time. */
+int afd_ffn_mailbox_take(afd_ffn_mailbox *mb, int32_t *slot, int32_t *T, int64_t timeout_us);
+/* Consumer: finish a taken slot: status AFD_OK -> done, a negative status -> failed. */
+int afd_ffn_mailbox_complete(afd_ffn_mailbox *mb, int32_t slot, int32_t status);
+/* Post / take / complete times of the slot's latest round: times_ns[3], 0 where not reached. */
+int afd_ffn_mailbox_times(afd_ffn_mailbox *mb, int32_t slot, int64_t *times_ns);
+
+typedef struct {
+  int64_t served;           /* micro-batches completed                                      */
+  int32_t status;           /* AFD_OK, or the first failure of the loop                      */
+  int32_t device_status;    /* afd_ffn_get_error of the handle when the loop ended           */
+  int32_t last_cuda_error;  /* cudaError_t behind an AFD_ERR_CUDA status, else 0             */
+  int32_t reserved;
+} afd_ffn_service_stats;
+
+/* Start the serving loop on its own host thread: for each slot taken from mb, copy its input
+ * to the device, run afd_ffn_forward on `stream`, copy the output back and complete the slot
+ * when that copy has landed.  Copies run on two streams of the service, so with two or more
+ * slots in flight the copies of one micro-batch overlap the layer of another.  The handle's
+ * H must equal the mailbox's and its T_max must be >= the mailbox's; the calling thread's
+ * current device must be the handle's.  While the service runs, the caller makes no other call
+ * on h.  After the first failure every later slot fails with the same status. */
+int afd_ffn_service_start(afd_ffn_handle *h, afd_ffn_mailbox *mb, void *stream, afd_ffn_service **out);
+/* Device timeline of a slot's latest micro-batch, from CUDA events the loop records (the slot
+ * must be done; call it before posting the slot again): ms[0] = service start -> H2D start, and
+ * from the H2D start: ms[1] H2D end, ms[2] layer start, ms[3] layer end, ms[4] D2H end.
+ * AFD_ERR_INVALID_ARG for a slot that is not done. */
+int afd_ffn_service_slot_timeline(afd_ffn_service *svc, int32_t slot, float *ms);
+/* Stop taking slots, let the ones in flight finish, fail the posted ones with AFD_ERR_STOPPED,
+ * release the service and fill *stats (may be NULL).  Returns stats.status. */
+int afd_ffn_service_stop(afd_ffn_service *svc, afd_ffn_service_stats *stats);
 
 #ifdef __cplusplus
 }

@@ -18,7 +18,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_strerror_covers_every_status():
-    for st in range(0, -8, -1):
+    for st in range(0, -10, -1):
         s = afd.afd_ffn_strerror(st)
         assert s and s != "unknown status"
     assert afd.afd_ffn_strerror(12345) == "unknown status"
@@ -88,3 +88,15 @@ def test_expert_parallel_calls_fail_fast_on_bad_arguments():
     assert afd.afd_ffn_combine_rows(A, None, A, A, 4, 2, 6, A) == afd.AFD_ERR_INVALID_ARG               # H % 4
     assert afd.afd_ffn_combine_rows(A, A + 4, A, A, 4, 2, 256, A) == afd.AFD_ERR_INVALID_ARG            # Ys align
     assert afd.afd_ffn_combine_rows(A, None, A, A, 0, 2, 256, A) == afd.AFD_OK                          # T = 0
+
+
+def test_service_calls_fail_fast_without_a_handle():
+    assert afd.afd_ffn_service_start(None, None)[0] == afd.AFD_ERR_INVALID_ARG
+    st, mb = afd.afd_ffn_mailbox_create(1, 4, 64, 0)
+    assert st == afd.AFD_OK
+    try:
+        assert afd.afd_ffn_service_start(None, mb)[0] == afd.AFD_ERR_INVALID_ARG
+    finally:
+        afd.afd_ffn_mailbox_destroy(mb)
+    assert afd.afd_ffn_service_stop(None)[0] == afd.AFD_ERR_INVALID_ARG
+    assert afd.afd_ffn_get_info(None)[0] == afd.AFD_ERR_INVALID_ARG
