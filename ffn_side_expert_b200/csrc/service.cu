@@ -5,9 +5,10 @@
 // "2. FFN Service").  Here the two sides meet in a mailbox of host buffers: the attention side
 // posts a micro-batch into a slot and later waits for the slot's output; the serving loop takes
 // slots in post order, copies the input to the device, runs afd_ffn_forward and copies the
-// output back.  With two or more slots in flight the attention of one micro-batch overlaps the
-// FFN of another (A/F 分离 page, section 深入推导, 微流水), and the host-to-device copy of one,
-// the layer of another and the device-to-host copy of a third run on three streams.
+// output back; a second thread completes each slot as soon as its output has landed.  With two
+// or more slots in flight the attention of one micro-batch overlaps the FFN of another (A/F 分离
+// page, section 深入推导, 微流水), and the host-to-device copy of one, the layer of another and
+// the device-to-host copy of a third run on three streams.
 //
 // Host code only; every step of the layer is afd_ffn_forward's kernels.  All waits are bounded.
 #include "afd_ffn.h"
@@ -259,17 +260,7 @@ int afd_ffn_mailbox_times(afd_ffn_mailbox* mb, int32_t slot, int64_t* times_ns) 
 // ------------------------------------------------------------------------ serving loop
 namespace {
 
-struct Landed {             // argument of the host function that completes a slot
-  afd_ffn_mailbox* mb = nullptr;
-  int32_t slot = 0;
-  std::atomic<int64_t>* served = nullptr;
-};
-
-void CUDART_CB on_output_landed(void* p) {
-  Landed* d = static_cast<Landed*>(p);
-  if (afd_ffn_mailbox_complete(d->mb, d->slot, AFD_OK) == AFD_OK)
-    d->served->fetch_add(1, std::memory_order_relaxed);
-}
+constexpr int64_t kLandNs = 60LL * 1000000000LL;   // give up on a micro-batch's output after 60 s
 
 }  // namespace
 
@@ -282,20 +273,30 @@ struct afd_ffn_service {
   std::unique_ptr<void*[]> din, dout;                 // per slot, device [T_max][H] bf16
   std::unique_ptr<cudaEvent_t[]> ev_h2d, ev_in, ev_start, ev_fwd, ev_out;   // timing events per slot
   cudaEvent_t ev_origin = nullptr;                     // recorded once when the loop is set up
-  std::unique_ptr<Landed[]> landed;
-  std::thread thread;
+  std::thread thread, completer;
   std::atomic<bool> stop{false};
   std::atomic<int64_t> served{0};
-  int32_t status = AFD_OK;          // written by the loop thread; read after join
+  std::atomic<int32_t> status{AFD_OK};         // first failure of the loop or the completer
+  std::atomic<int32_t> last_cuda_error{0};
   int32_t device_status = AFD_OK;
-  int32_t last_cuda_error = 0;
+  // slots whose D2H is enqueued, oldest first; the completer finishes them in this order
+  std::mutex fl_mu;
+  std::condition_variable fl_cv;
+  std::unique_ptr<int32_t[]> in_flight;        // ring of n_slots entries
+  uint64_t fl_head = 0, fl_tail = 0;           // under fl_mu
+  bool loop_done = false;                      // under fl_mu: no more slots will be enqueued
 };
 
 namespace {
 
 int note_cuda(afd_ffn_service* v, cudaError_t e) {
-  v->last_cuda_error = static_cast<int32_t>(e);
+  v->last_cuda_error.store(static_cast<int32_t>(e));
   return AFD_ERR_CUDA;
+}
+
+void fail(afd_ffn_service* v, int32_t st) {
+  int32_t ok = AFD_OK;
+  v->status.compare_exchange_strong(ok, st);
 }
 
 #define SVC_CUDA(v, call)                              \
@@ -305,9 +306,9 @@ int note_cuda(afd_ffn_service* v, cudaError_t e) {
   } while (0)
 
 // Enqueue one micro-batch: H2D on copy_in, the layer on the caller's stream, D2H on copy_out,
-// then a host function that completes the slot once the output has landed.  A slot is re-posted
-// only after it completed, so its buffers are free again; the event waits say so to the device
-// as well.
+// and hand the slot to the completer, which completes it once the D2H has landed.  A slot is
+// re-posted only after it completed, so its buffers are free again; the event waits say so to
+// the device as well.
 int serve_one(afd_ffn_service* v, int32_t slot, int32_t T) {
   Slot& s = v->mb->slots[slot];
   const size_t bytes = static_cast<size_t>(T) * static_cast<size_t>(v->mb->H) * 2;
@@ -320,15 +321,50 @@ int serve_one(afd_ffn_service* v, int32_t slot, int32_t T) {
   SVC_CUDA(v, cudaEventRecord(v->ev_start[slot], v->stream));
   const int st = afd_ffn_forward(v->h, v->din[slot], T, v->dout[slot], v->stream);
   if (st != AFD_OK) {
-    if (st == AFD_ERR_CUDA) v->last_cuda_error = afd_ffn_last_cuda_error(v->h);
+    if (st == AFD_ERR_CUDA) v->last_cuda_error.store(afd_ffn_last_cuda_error(v->h));
     return st;
   }
   SVC_CUDA(v, cudaEventRecord(v->ev_fwd[slot], v->stream));
   SVC_CUDA(v, cudaStreamWaitEvent(v->copy_out, v->ev_fwd[slot], 0));
   if (bytes) SVC_CUDA(v, cudaMemcpyAsync(s.out, v->dout[slot], bytes, cudaMemcpyDeviceToHost, v->copy_out));
   SVC_CUDA(v, cudaEventRecord(v->ev_out[slot], v->copy_out));
-  SVC_CUDA(v, cudaLaunchHostFunc(v->copy_out, on_output_landed, &v->landed[slot]));
+  {
+    std::lock_guard<std::mutex> g(v->fl_mu);
+    v->in_flight[v->fl_tail++ % static_cast<uint64_t>(v->mb->n_slots)] = slot;
+  }
+  v->fl_cv.notify_one();
   return AFD_OK;
+}
+
+// The completer: for each enqueued slot in order, poll the event after its D2H and complete the
+// slot as soon as the output is in host memory.  Polling costs this thread's core while
+// micro-batches are in flight and gives the attention side the output within microseconds; it
+// sleeps when nothing is in flight.
+void complete_loop(afd_ffn_service* v) {
+  cudaSetDevice(v->device);
+  for (;;) {
+    int32_t slot;
+    {
+      std::unique_lock<std::mutex> lk(v->fl_mu);
+      v->fl_cv.wait(lk, [&] { return v->fl_head < v->fl_tail || v->loop_done; });
+      if (v->fl_head == v->fl_tail) return;          // the loop has ended and nothing is left
+      slot = v->in_flight[v->fl_head++ % static_cast<uint64_t>(v->mb->n_slots)];
+    }
+    cudaError_t e = cudaErrorNotReady;
+    const int64_t give_up = now_ns() + kLandNs;
+    for (int n = 0;; ++n) {
+      e = cudaEventQuery(v->ev_out[slot]);
+      if (e != cudaErrorNotReady || now_ns() > give_up) break;
+      if (n < 256) cpu_relax(); else std::this_thread::yield();
+    }
+    if (e == cudaSuccess) {
+      if (afd_ffn_mailbox_complete(v->mb, slot, AFD_OK) == AFD_OK) v->served.fetch_add(1);
+    } else {
+      const int32_t st = e == cudaErrorNotReady ? AFD_ERR_TIMEOUT : note_cuda(v, e);
+      fail(v, st);
+      afd_ffn_mailbox_complete(v->mb, slot, st);
+    }
+  }
 }
 
 void drain(afd_ffn_service* v) {
@@ -337,27 +373,37 @@ void drain(afd_ffn_service* v) {
   cudaStreamSynchronize(v->copy_out);
 }
 
+void end_completer(afd_ffn_service* v) {
+  {
+    std::lock_guard<std::mutex> g(v->fl_mu);
+    v->loop_done = true;
+  }
+  v->fl_cv.notify_one();
+  if (v->completer.joinable()) v->completer.join();
+}
+
 void serve_loop(afd_ffn_service* v) {
-  if (cudaSetDevice(v->device) != cudaSuccess) v->status = AFD_ERR_NO_DEVICE;
+  if (cudaSetDevice(v->device) != cudaSuccess) fail(v, AFD_ERR_NO_DEVICE);
   while (!v->stop.load(std::memory_order_acquire)) {
     int32_t slot = 0, T = 0;
     if (take_slot(v->mb, &slot, &T, kPollUs, &v->stop) != AFD_OK) continue;
-    int st = v->status;
+    int st = v->status.load();
     if (st == AFD_OK && (st = serve_one(v, slot, T)) != AFD_OK) {
-      v->status = st;
+      fail(v, st);
       drain(v);     // nothing of this slot may still be reading or writing its buffers
     }
     if (st != AFD_OK) afd_ffn_mailbox_complete(v->mb, slot, st);
   }
+  end_completer(v);   // every enqueued slot is completed before this returns
   drain(v);
   const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess && v->status == AFD_OK) v->status = note_cuda(v, e);
+  if (e != cudaSuccess) fail(v, note_cuda(v, e));
   // posted but never taken
   int32_t slot = 0, T = 0;
   while (afd_ffn_mailbox_take(v->mb, &slot, &T, 0) == AFD_OK) afd_ffn_mailbox_complete(v->mb, slot, AFD_ERR_STOPPED);
-  // taken, but the host function never ran (the stream failed after the enqueue)
-  for (int32_t i = 0; i < v->mb->n_slots; ++i)
-    afd_ffn_mailbox_complete(v->mb, i, v->status != AFD_OK ? v->status : AFD_ERR_CUDA);  // no-op unless taken
+  // taken but never completed (cannot happen after the completer drained; kept as a guard)
+  const int32_t end_st = v->status.load() != AFD_OK ? v->status.load() : AFD_ERR_CUDA;
+  for (int32_t i = 0; i < v->mb->n_slots; ++i) afd_ffn_mailbox_complete(v->mb, i, end_st);   // no-op unless taken
   v->device_status = afd_ffn_get_error(v->h);
 }
 
@@ -384,8 +430,8 @@ int setup(afd_ffn_service* v) {
   v->dout.reset(new (std::nothrow) void*[n]());
   std::unique_ptr<cudaEvent_t[]>* const evsets[] = {&v->ev_h2d, &v->ev_in, &v->ev_start, &v->ev_fwd, &v->ev_out};
   for (auto* evs : evsets) evs->reset(new (std::nothrow) cudaEvent_t[n]());
-  v->landed.reset(new (std::nothrow) Landed[n]);
-  if (!v->din || !v->dout || !v->ev_h2d || !v->ev_in || !v->ev_start || !v->ev_fwd || !v->ev_out || !v->landed)
+  v->in_flight.reset(new (std::nothrow) int32_t[n]());
+  if (!v->din || !v->dout || !v->ev_h2d || !v->ev_in || !v->ev_start || !v->ev_fwd || !v->ev_out || !v->in_flight)
     return AFD_ERR_INVALID_ARG;
   SVC_CUDA(v, cudaStreamCreateWithFlags(&v->copy_in, cudaStreamNonBlocking));
   SVC_CUDA(v, cudaStreamCreateWithFlags(&v->copy_out, cudaStreamNonBlocking));
@@ -395,9 +441,6 @@ int setup(afd_ffn_service* v) {
     SVC_CUDA(v, cudaMalloc(&v->din[i], bytes));
     SVC_CUDA(v, cudaMalloc(&v->dout[i], bytes));
     for (auto* evs : evsets) SVC_CUDA(v, cudaEventCreate(&(*evs)[i]));
-    v->landed[i].mb = v->mb;
-    v->landed[i].slot = i;
-    v->landed[i].served = &v->served;
   }
   return AFD_OK;
 }
@@ -434,10 +477,17 @@ int afd_ffn_service_start(afd_ffn_handle* h, afd_ffn_mailbox* mb, void* stream, 
     return st;
   }
   try {
-    v->thread = std::thread(serve_loop, v);
+    v->completer = std::thread(complete_loop, v);
   } catch (...) {
     release(v);
     return AFD_ERR_UNSUPPORTED;     // no host thread could be started
+  }
+  try {
+    v->thread = std::thread(serve_loop, v);
+  } catch (...) {
+    end_completer(v);
+    release(v);
+    return AFD_ERR_UNSUPPORTED;
   }
   *out = v;
   return AFD_OK;
@@ -448,12 +498,12 @@ int afd_ffn_service_stop(afd_ffn_service* v, afd_ffn_service_stats* stats) {
   v->stop.store(true, std::memory_order_release);
   notify(v->mb);
   if (v->thread.joinable()) v->thread.join();
-  const int32_t status = v->status;
+  const int32_t status = v->status.load();
   if (stats) {
     stats->served = v->served.load();
     stats->status = status;
     stats->device_status = v->device_status;
-    stats->last_cuda_error = v->last_cuda_error;
+    stats->last_cuda_error = v->last_cuda_error.load();
     stats->reserved = 0;
   }
   release(v);
