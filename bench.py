@@ -11,6 +11,12 @@ not sharded: no collective on the data path); value = total tokens of all ranks 
 slowest rank's time.  --impl reference times the fp64 CPU oracle on a bounded sample of the
 same workload instead (the reference arm).
 
+    python bench.py --period [--config dsv3_256]
+
+measures the FFN-service micro-pipeline instead: a host attention stub of set duration t_a
+feeds the library's serving loop with one or two micro-batches in flight, and the period is
+compared with the A/F split's model max(t_a, t_f) + t_comm and with t_a + t_f on one device.
+
 Prints one JSON line (rank 0).
 """
 from __future__ import annotations
@@ -558,6 +564,21 @@ def pipeline_period(layer, hidden_host, T, t_a_ms, n_slots, rounds, ref_out=None
     return period, mismatches, stats, parts
 
 
+def period_models(t_a, t_f, t_h2d, t_d2h, slots) -> dict:
+    """Steady-state period of the A/F micro-pipeline, ms per micro-batch.
+
+    page: the A/F 分离 page's model (section 深入推导, 微流水), max(t_a, t_f) + t_comm with
+    micro-batches overlapped, t_a + t_f + t_comm without (one slot).
+    cycle: a bound for the serving loop, whose copies overlap the layer.  The attention side
+    and the layer each serve one micro-batch at a time, and one slot's micro-batch goes round
+    attention -> H2D -> layer -> D2H before the slot is used again, so with `slots` of them in
+    flight the period is at least max(t_a, t_f, (t_a + t_h2d + t_f + t_d2h) / slots)."""
+    t_comm = t_h2d + t_d2h
+    page = (max(t_a, t_f) if slots > 1 else t_a + t_f) + t_comm
+    cycle = max(t_a, t_f, (t_a + t_h2d + t_f + t_d2h) / slots)
+    return {"page": page, "cycle": cycle, "colocated": t_a + t_f}
+
+
 def run_period(args) -> dict:
     """The micro-pipeline period of the A/F split (A/F 分离 page, section 深入推导, 微流水): the
     steady-state period with the attention of one micro-batch overlapping the FFN of another,
@@ -605,9 +626,13 @@ def run_period(args) -> dict:
             bad += mism
             if st.status != afd.AFD_OK or st.device_status != afd.AFD_OK:
                 raise afd.AfdError(st.status or st.device_status, "FFN service")
-            model = (max(t_a, t_f) if slots > 1 else t_a + t_f) + t_comm
+            m = period_models(t_a, t_f, t_h2d, t_d2h, slots)
+            # the bound again with the copy and layer times this point measured in the loop
+            m_in_loop = period_models(t_a, parts["layer_ms"], parts["h2d_ms"], parts["d2h_after_layer_ms"], slots)
             points.append({"t_a_ms": round(t_a, 4), "slots": slots, "period_ms": round(period, 4),
-                           "model_ms": round(model, 4), "colocated_ms": round(t_a + t_f, 4),
+                           "model_ms": round(m["page"], 4), "cycle_bound_ms": round(m["cycle"], 4),
+                           "cycle_bound_in_loop_ms": round(m_in_loop["cycle"], 4),
+                           "colocated_ms": round(t_a + t_f, 4),
                            "period_over_colocated": round(period / (t_a + t_f), 3), **parts})
     return {
         "metric": "FFN-service micro-pipeline period", "unit": "ms", "higher_is_better": False,
@@ -615,7 +640,10 @@ def run_period(args) -> dict:
                    "n_shared": cfg.S, "weights": cfg.dtype, "attention": "host stub, busy t_a per micro-batch",
                    "link": "PCIe host<->device copies (pinned)", "rounds": rounds},
         "t_f_ms": round(t_f, 4), "t_comm_ms": {"h2d": round(t_h2d, 4), "d2h": round(t_d2h, 4), "sum": round(t_comm, 4)},
-        "models": {"slots=1": "t_a + t_f + t_comm", "slots=2": "max(t_a, t_f) + t_comm", "colocated": "t_a + t_f"},
+        "models": {"model_ms": "slots=1: t_a + t_f + t_comm; slots=2: max(t_a, t_f) + t_comm",
+                   "cycle_bound_ms": "max(t_a, t_f, (t_a + t_h2d + t_f + t_d2h) / slots)",
+                   "cycle_bound_in_loop_ms": "the same with the H2D, layer and D2H times measured in the loop",
+                   "colocated_ms": "t_a + t_f"},
         "points": points, "outputs_bit_equal_to_forward": bad == 0,
     }
 
