@@ -81,6 +81,7 @@ _SIGNATURES = {
     "afd_ffn_combine_rows": (ctypes.c_int, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "afd_ffn_rows_error": (ctypes.c_int, []),
     "afd_ffn_get_info": (ctypes.c_int, [_P, ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(ctypes.c_int32)]),
+    "afd_ffn_check_bounded_wait": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int64)]),
     "afd_ffn_mailbox_create": (ctypes.c_int, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_void_p)]),
     "afd_ffn_mailbox_destroy": (None, [_P]),
     "afd_ffn_mailbox_input": (_P, [_P, _I]),
@@ -249,6 +250,13 @@ def afd_ffn_combine_rows(Y, Ys, topk_w, pos, T, k, H, out, stream=None) -> int:
 
 def afd_ffn_rows_error() -> int:
     return _lib.afd_ffn_rows_error()
+
+
+def afd_ffn_check_bounded_wait():
+    """Returns (status, SM cycles the wait took); AFD_ERR_DEVICE_TIMEOUT is the expected status."""
+    cycles = ctypes.c_int64(0)
+    st = _lib.afd_ffn_check_bounded_wait(ctypes.byref(cycles))
+    return st, cycles.value
 
 
 def afd_ffn_get_info(h):

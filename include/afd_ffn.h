@@ -240,6 +240,15 @@ int afd_ffn_combine_rows(const float *Y, const float *Ys, const float *topk_w, c
  * since the last check (the word is cleared), else AFD_OK. */
 int afd_ffn_rows_error(void);
 
+/* Self-check of the device's bounded waits.  One thread waits, through the same bounded wait
+ * the GEMM roles use, on an mbarrier that no thread arrives on; the wait must give up after its
+ * limit (about 2 s of SM clock) and record the timeout bit, and the kernel then returns.
+ * Synchronous (the device is synchronised), on the current device.  Returns
+ * AFD_ERR_DEVICE_TIMEOUT when the wait gave up and the bit reached the host (the expected
+ * result), AFD_OK if the wait completed, AFD_ERR_CUDA / AFD_ERR_NO_DEVICE on failure.
+ * *waited_cycles (may be NULL) receives the SM cycles the wait took. */
+int afd_ffn_check_bounded_wait(int64_t *waited_cycles);
+
 /* The configuration and device of a handle (host only; either output may be NULL). */
 int afd_ffn_get_info(const afd_ffn_handle *h, afd_ffn_cfg *cfg, int32_t *device);
 

@@ -100,3 +100,10 @@ def test_service_calls_fail_fast_without_a_handle():
         afd.afd_ffn_mailbox_destroy(mb)
     assert afd.afd_ffn_service_stop(None)[0] == afd.AFD_ERR_INVALID_ARG
     assert afd.afd_ffn_get_info(None)[0] == afd.AFD_ERR_INVALID_ARG
+
+
+def test_bounded_wait_check_needs_a_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present: the GPU test covers the call")
+    assert afd.afd_ffn_check_bounded_wait()[0] == afd.AFD_ERR_NO_DEVICE
