@@ -579,6 +579,19 @@ def period_models(t_a, t_f, t_h2d, t_d2h, slots) -> dict:
     return {"page": page, "cycle": cycle, "colocated": t_a + t_f}
 
 
+def period_point(t_a, slots, period, parts, t_f, t_h2d, t_d2h) -> dict:
+    """One measured point of --period with its models: the page's, the cycle bound from the
+    isolated layer and copy times, and the cycle bound again from the times measured in the
+    loop (parts: the breakdown pipeline_period returns)."""
+    m = period_models(t_a, t_f, t_h2d, t_d2h, slots)
+    m_in_loop = period_models(t_a, parts["layer_ms"], parts["h2d_ms"], parts["d2h_after_layer_ms"], slots)
+    return {"t_a_ms": round(t_a, 4), "slots": slots, "period_ms": round(period, 4),
+            "model_ms": round(m["page"], 4), "cycle_bound_ms": round(m["cycle"], 4),
+            "cycle_bound_in_loop_ms": round(m_in_loop["cycle"], 4),
+            "colocated_ms": round(m["colocated"], 4),
+            "period_over_colocated": round(period / m["colocated"], 3), **parts}
+
+
 def run_period(args) -> dict:
     """The micro-pipeline period of the A/F split (A/F 分离 page, section 深入推导, 微流水): the
     steady-state period with the attention of one micro-batch overlapping the FFN of another,
@@ -626,14 +639,7 @@ def run_period(args) -> dict:
             bad += mism
             if st.status != afd.AFD_OK or st.device_status != afd.AFD_OK:
                 raise afd.AfdError(st.status or st.device_status, "FFN service")
-            m = period_models(t_a, t_f, t_h2d, t_d2h, slots)
-            # the bound again with the copy and layer times this point measured in the loop
-            m_in_loop = period_models(t_a, parts["layer_ms"], parts["h2d_ms"], parts["d2h_after_layer_ms"], slots)
-            points.append({"t_a_ms": round(t_a, 4), "slots": slots, "period_ms": round(period, 4),
-                           "model_ms": round(m["page"], 4), "cycle_bound_ms": round(m["cycle"], 4),
-                           "cycle_bound_in_loop_ms": round(m_in_loop["cycle"], 4),
-                           "colocated_ms": round(t_a + t_f, 4),
-                           "period_over_colocated": round(period / (t_a + t_f), 3), **parts})
+            points.append(period_point(t_a, slots, period, parts, t_f, t_h2d, t_d2h))
     return {
         "metric": "FFN-service micro-pipeline period", "unit": "ms", "higher_is_better": False,
         "config": {"workload": workload_label(args), "T": T, "H": H, "E": cfg.E, "k": cfg.k, "I": cfg.I,

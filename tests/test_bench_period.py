@@ -40,3 +40,16 @@ def test_cycle_bound_never_exceeds_the_page_model():
             m = bench.period_models(t_a, t_f, h, d, slots)
             assert m["cycle"] <= m["page"] + 1e-12
             assert m["cycle"] >= max(t_a, t_f) - 1e-12
+
+
+def test_a_measured_point_carries_its_models():
+    # the parts of the balanced two-slot point measured at the T=256 decode shape
+    parts = {"post_to_take_ms": 0.0131, "take_to_landed_ms": 3.846, "period_mean_ms": 3.701,
+             "h2d_ms": 0.096, "h2d_end_to_layer_ms": 0.008, "layer_ms": 3.501, "layer_gap_ms": 0.1712,
+             "d2h_after_layer_ms": 0.079, "host_overhead_ms": 0.012}
+    p = bench.period_point(3.4939, 2, 3.697, parts, 3.4939, 0.0842, 0.0705)
+    assert p["model_ms"] == pytest.approx(3.4939 + 0.0842 + 0.0705, abs=1e-4)
+    assert p["cycle_bound_in_loop_ms"] == pytest.approx((3.4939 + 0.096 + 3.501 + 0.079) / 2, abs=1e-4)
+    assert p["colocated_ms"] == pytest.approx(2 * 3.4939, abs=1e-4)
+    assert p["period_over_colocated"] == pytest.approx(3.697 / (2 * 3.4939), abs=1e-3)
+    assert p["layer_gap_ms"] == 0.1712 and p["slots"] == 2
