@@ -256,8 +256,10 @@ int afd_ffn_get_info(const afd_ffn_handle *h, afd_ffn_cfg *cfg, int32_t *device)
  * The FFN side of an A/F split runs a loop per layer: take the activations the attention side
  * sent, run the layer, send the output back (vLLM AFD Plugin page, section 系統架構, "2. FFN
  * Service").  With several micro-batches in flight the attention of one overlaps the FFN of
- * another, so the steady-state period is max(t_a, t_f) + t_comm instead of t_a + t_f when both
- * share a device (A/F 分离 page, section 深入推导, 微流水).
+ * another: the A/F 分离 page (section 深入推导, 微流水) puts the steady-state period at
+ * max(t_a, t_f) + t_comm instead of t_a + t_f on one device.  This loop also overlaps the
+ * copies with the layer, so with n slots in flight its period is bounded below by
+ * max(t_a, t_f, (t_a + t_h2d + t_f + t_d2h) / n).
  *
  * The mailbox is the connector between the two sides on one host: n_slots slots, each an input
  * buffer [T_max][H] bf16 (the hidden states of one micro-batch) and an output buffer of the
@@ -303,19 +305,23 @@ int afd_ffn_mailbox_times(afd_ffn_mailbox *mb, int32_t slot, int64_t *times_ns);
 
 typedef struct {
   int64_t served;           /* micro-batches completed                                      */
-  int32_t status;           /* AFD_OK, or the first failure of the loop                      */
+  int32_t status;           /* AFD_OK, or the first failure of the loop or the completer     */
   int32_t device_status;    /* afd_ffn_get_error of the handle when the loop ended           */
   int32_t last_cuda_error;  /* cudaError_t behind an AFD_ERR_CUDA status, else 0             */
   int32_t reserved;
 } afd_ffn_service_stats;
 
-/* Start the serving loop on its own host thread: for each slot taken from mb, copy its input
- * to the device, run afd_ffn_forward on `stream`, copy the output back and complete the slot
- * when that copy has landed.  Copies run on two streams of the service, so with two or more
- * slots in flight the copies of one micro-batch overlap the layer of another.  The handle's
- * H must equal the mailbox's and its T_max must be >= the mailbox's; the calling thread's
- * current device must be the handle's.  While the service runs, the caller makes no other call
- * on h.  After the first failure every later slot fails with the same status. */
+/* Start the serving loop on two host threads.  The loop thread takes each slot from mb and
+ * enqueues its micro-batch: the input copied to the device, afd_ffn_forward on `stream`, the
+ * output copied back.  The copies run on two streams of the service, so with two or more slots
+ * in flight the copies of one micro-batch overlap the layer of another.  The completer thread
+ * polls the event after each in-flight slot's copy back, in order, and completes the slot as
+ * soon as its output has landed.  It keeps one core busy while micro-batches are in flight and
+ * sleeps otherwise.  An output that has not landed after 60 s fails its slot with
+ * AFD_ERR_TIMEOUT.
+ * The handle's H must equal the mailbox's and its T_max must be >= the mailbox's; the calling
+ * thread's current device must be the handle's.  While the service runs, the caller makes no
+ * other call on h.  After the first failure every later slot fails with the same status. */
 int afd_ffn_service_start(afd_ffn_handle *h, afd_ffn_mailbox *mb, void *stream, afd_ffn_service **out);
 /* Device timeline of a slot's latest micro-batch, from CUDA events the loop records (the slot
  * must be done; call it before posting the slot again): ms[0] = service start -> H2D start, and
