@@ -358,6 +358,8 @@ class AfdFfn:
 
     def close(self):
         if getattr(self, "h", None):
+            if getattr(self, "_served_by", 0):
+                raise RuntimeError("an FfnService is still running on this layer: stop it first")
             afd_ffn_destroy(self.h)
             self.h = None
 

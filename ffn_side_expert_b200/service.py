@@ -41,6 +41,7 @@ class Mailbox:
         if st != AFD_OK:
             raise AfdError(st, "afd_ffn_mailbox_create")
         self.n_slots, self.T_max, self.H = n_slots, T_max, H
+        self._served_by = 0          # running FfnService loops on this mailbox
         self._in = [_host_view(afd_ffn_mailbox_input(self.mb, i), T_max, H) for i in range(n_slots)]
         self._out = [_host_view(afd_ffn_mailbox_output(self.mb, i), T_max, H) for i in range(n_slots)]
 
@@ -87,6 +88,8 @@ class Mailbox:
 
     def close(self) -> None:
         if getattr(self, "mb", None):
+            if self._served_by:
+                raise RuntimeError("an FfnService is still running on this mailbox: stop it first")
             self._in, self._out = [], []
             afd_ffn_mailbox_destroy(self.mb)
             self.mb = None
@@ -103,11 +106,17 @@ class FfnService:
     native thread.  While it runs, make no other call on the layer."""
 
     def __init__(self, layer, mailbox: Mailbox, stream=None):
-        st, self.svc = afd_ffn_service_start(layer.h, mailbox.mb, stream)
+        self.svc = None
+        if not getattr(layer, "h", None) or not getattr(mailbox, "mb", None):
+            raise ValueError("the layer and the mailbox must be open")
+        st, svc = afd_ffn_service_start(layer.h, mailbox.mb, stream)
         if st != AFD_OK:
             raise AfdError(st, "afd_ffn_service_start")
-        self.layer, self.mailbox = layer, mailbox
+        self.svc, self.layer, self.mailbox = svc, layer, mailbox
         self.stats = None
+        # neither may be closed while the loop runs on them
+        mailbox._served_by += 1
+        layer._served_by = getattr(layer, "_served_by", 0) + 1
 
     def timeline(self, slot: int):
         """Device timeline (ms) of the slot's latest micro-batch: service start -> H2D start, then
@@ -123,6 +132,8 @@ class FfnService:
         if self.svc:
             _, self.stats = afd_ffn_service_stop(self.svc)
             self.svc = None
+            self.mailbox._served_by -= 1
+            self.layer._served_by -= 1
         return self.stats
 
     def __del__(self):

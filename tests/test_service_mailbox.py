@@ -138,3 +138,48 @@ def test_write_input_copies_rows_and_checks_them(mb):
     for bad in (rows.float(), rows.t(), rows[:, :32].contiguous(), torch.zeros(17, 64, dtype=torch.bfloat16)):
         with pytest.raises(ValueError):
             mb.write_input(0, bad)
+
+
+class _NoDeviceLayer(afd.AfdFfn):
+    """An AfdFfn shell with a stand-in handle value: only its close guard is exercised."""
+
+    def __init__(self):
+        self.h = 99
+
+
+def test_a_running_service_keeps_its_layer_and_mailbox_open(monkeypatch):
+    from ffn_side_expert_b200 import service
+    stopped = []
+    monkeypatch.setattr(service, "afd_ffn_service_start", lambda h, mb, stream=None: (afd.AFD_OK, 4242))
+    monkeypatch.setattr(service, "afd_ffn_service_stop",
+                        lambda svc: (stopped.append(svc), (afd.AFD_OK, afd.afd_ffn_service_stats(served=3)))[1])
+    layer, m = _NoDeviceLayer(), Mailbox(2, 4, 64, pinned=False)
+    try:
+        svc = service.FfnService(layer, m)
+        with pytest.raises(RuntimeError):
+            m.close()
+        with pytest.raises(RuntimeError):
+            layer.close()
+        assert svc.stop().served == 3 and stopped == [4242]
+        assert svc.stop().served == 3 and stopped == [4242]          # a second stop does nothing
+        assert m._served_by == 0 and layer._served_by == 0
+        m.close()                                                      # allowed once stopped
+    finally:
+        layer.h = None                                                 # nothing real to destroy
+        m.close()
+
+
+def test_a_service_that_fails_to_start_holds_nothing(monkeypatch):
+    from ffn_side_expert_b200 import service
+    monkeypatch.setattr(service, "afd_ffn_service_start", lambda h, mb, stream=None: (afd.AFD_ERR_INVALID_ARG, None))
+    layer, m = _NoDeviceLayer(), Mailbox(2, 4, 64, pinned=False)
+    try:
+        with pytest.raises(afd.AfdError):
+            service.FfnService(layer, m)
+        assert m._served_by == 0 and getattr(layer, "_served_by", 0) == 0
+        m.close()
+        with pytest.raises(ValueError):
+            service.FfnService(layer, m)                               # a closed mailbox
+    finally:
+        layer.h = None
+        m.close()
