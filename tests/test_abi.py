@@ -107,3 +107,26 @@ def test_bounded_wait_check_needs_a_device():
     if torch.cuda.is_available():
         pytest.skip("a device is present: the GPU test covers the call")
     assert afd.afd_ffn_check_bounded_wait()[0] == afd.AFD_ERR_NO_DEVICE
+
+
+def _declared_arities(header=afd.HEADER_PATH):
+    import re
+    with open(header) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(afd_ffn_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = " ".join(m.group(2).split())
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every declared entry point is bound with as many ctypes arguments as the header gives
+    it, and with a result type (None only for the void ones)."""
+    arity = _declared_arities()
+    assert set(arity) == set(afd.declared_functions())
+    for name, n in arity.items():
+        res, args = afd._SIGNATURES[name]
+        assert len(args) == n, (name, len(args), n)
+    for name in ("afd_ffn_destroy", "afd_ffn_mailbox_destroy"):
+        assert afd._SIGNATURES[name][0] is None
