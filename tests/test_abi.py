@@ -109,15 +109,37 @@ def test_bounded_wait_check_needs_a_device():
     assert afd.afd_ffn_check_bounded_wait()[0] == afd.AFD_ERR_NO_DEVICE
 
 
-def _declared_arities(header=afd.HEADER_PATH):
+def _declared_params(header=afd.HEADER_PATH):
+    """name -> list of parameter kinds ('ptr', 'i32', 'i64', 'f32') from include/afd_ffn.h."""
     import re
     with open(header) as f:
         text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
     out = {}
     for m in re.finditer(r"\b(afd_ffn_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
         params = " ".join(m.group(2).split())
-        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+        kinds = []
+        for p in ([] if params in ("", "void") else params.split(",")):
+            if "*" in p:
+                kinds.append("ptr")
+            elif "int64_t" in p:
+                kinds.append("i64")
+            elif "float" in p:
+                kinds.append("f32")
+            else:
+                assert re.search(r"\b(int32_t|int)\b", p), p
+                kinds.append("i32")
+        out[m.group(1)] = kinds
     return out
+
+
+def _kind(ct):
+    if ct in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(ct, type(ctypes.POINTER(ctypes.c_int))):
+        return "ptr"
+    return {ctypes.c_int32: "i32", ctypes.c_int: "i32", ctypes.c_int64: "i64", ctypes.c_float: "f32"}[ct]
+
+
+def _declared_arities(header=afd.HEADER_PATH):
+    return {k: len(v) for k, v in _declared_params(header).items()}
 
 
 def test_binding_signatures_match_the_header():
@@ -130,3 +152,9 @@ def test_binding_signatures_match_the_header():
         assert len(args) == n, (name, len(args), n)
     for name in ("afd_ffn_destroy", "afd_ffn_mailbox_destroy"):
         assert afd._SIGNATURES[name][0] is None
+
+
+def test_binding_argument_kinds_match_the_header():
+    for name, kinds in _declared_params().items():
+        _, args = afd._SIGNATURES[name]
+        assert [_kind(a) for a in args] == kinds, name
