@@ -30,7 +30,7 @@ def _weights():
     return Wr, experts
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, tokens=TOKENS):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -38,12 +38,16 @@ def _worker(rank, world, port, q):
         from oracle import moe
         Wr, experts = _weights()
         el = E // world
-        hidden = torch.from_numpy(np.random.default_rng(100 + rank).normal(0, 1, (TOKENS[rank], H)))
+        hidden = torch.from_numpy(np.random.default_rng(100 + rank).normal(0, 1, (tokens[rank], H)))
         backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[rank * el:(rank + 1) * el],
                                     shared=experts[E])
         ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
         out = ep.forward(hidden)
         from oracle import comm
+        if tokens[rank] == 0:                             # an empty micro-batch still takes part
+            assert tuple(out.shape) == (0, H)
+            q.put((rank, 0.0, 0.0, ep.last_wire, 0))
+            return
         idx = moe.route(hidden.numpy(), Wr, None, K)[1]
         account = comm.element_bytes(idx, H, 8)          # the oracle's per-direction account
         ref = moe.forward(hidden.numpy(), Wr, None, lambda e: {"w13": experts[e][0], "w2": experts[e][1]},
@@ -53,26 +57,34 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_ranks_match_the_single_process_layer():
+def _run(tokens, port):
+    world = len(tokens)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29600 + os.getpid() % 1000
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, tokens)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(180)
         assert p.exitcode == 0
-    res = sorted(q.get(timeout=10) for _ in range(2))
+    res = sorted(q.get(timeout=10) for _ in range(world))
     for rank, err, scale, wire, account in res:
         assert err <= 1e-12 * max(scale, 1.0), (rank, err)
         # every token sends k rows to the experts' ranks and gets k rows back
-        assert wire.tokens == TOKENS[rank]
-        assert wire.dispatch_sent == TOKENS[rank] * K * H * 8          # float64 rows in this test
+        assert wire.tokens == tokens[rank]
+        assert wire.dispatch_sent == tokens[rank] * K * H * 8          # float64 rows in this test
         assert wire.dispatch_sent == account                           # = the oracle's element account
     sent = sum(r[3].dispatch_sent for r in res)
     back = sum(r[3].combine_sent for r in res)
     assert sent == back                                                # the same rows return
+
+
+def test_two_ranks_match_the_single_process_layer():
+    _run(TOKENS, 29600 + os.getpid() % 1000)
+
+
+def test_four_ranks_with_an_empty_and_a_one_token_micro_batch():
+    _run({0: 7, 1: 0, 2: 13, 3: 1}, 28600 + os.getpid() % 1000)
 
 
 def test_block_tables_regroup_and_restore():
