@@ -113,3 +113,45 @@ def test_block_tables_interleave_sources_per_expert():
         grouped[d:d + n] = received[s:s + n]
     assert grouped.tolist() == [10, 20, 11, 21]        # expert 0 rows from both sources first
     assert per_expert.tolist() == [2, 2]
+
+
+def _leaving_worker(rank, world, port, q):
+    """Rank 1 leaves between steps (after the group is up, before the next forward); rank 0's
+    next forward must end with an error from the group's short timeout, not hang."""
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    dist.barrier()
+    if rank == 1:
+        os._exit(0)                                   # leaves without taking the next step
+    from ep_support import OracleRowsBackend
+    Wr, experts = _weights()
+    backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[:E // world], shared=experts[E])
+    ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
+    hidden = torch.from_numpy(np.random.default_rng(3).normal(0, 1, (6, H)))
+    t0 = time.monotonic()
+    try:
+        ep.forward(hidden)
+        q.put(("no error", time.monotonic() - t0))
+    except Exception as e:                            # the exchange reports the missing peer
+        q.put((type(e).__name__, time.monotonic() - t0))
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_others_step_with_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 27600 + os.getpid() % 1000
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        outcome, seconds = q.get(timeout=90)
+    finally:
+        for p in procs:
+            p.join(30)
+            if p.is_alive():
+                p.kill()                              # this test's own child, by handle
+    assert outcome != "no error"
+    assert seconds < 60
