@@ -20,6 +20,7 @@ the exchange can be exercised on CPU ranks.
 """
 from __future__ import annotations
 
+import datetime
 from dataclasses import dataclass
 
 import torch
@@ -70,6 +71,14 @@ class WireBytes:
     combine_sent: int       # expert outputs sent back (fp32 rows)
     combine_remote: int
     tokens: int
+
+
+class PeerLost(RuntimeError):
+    """A rank of the group did not reach this step: found on the host, before any exchange."""
+
+    def __init__(self, step: int, missing: list):
+        self.step, self.missing = step, missing
+        super().__init__(f"ranks {missing} did not reach step {step}")
 
 
 class CudaRowsBackend:
@@ -148,10 +157,17 @@ class ExpertParallelFfn:
 
     Every rank calls forward() with its own micro-batch (the same T on all ranks is not
     required).  `backend` defaults to CudaRowsBackend built from the arguments.
+
+    liveness: optional torch.distributed Store that every rank of the group reaches.  With it,
+    each forward first checks on the host that every rank has reached the same step (each
+    rank sets its key, then waits up to liveness_timeout_s for the others').  A rank that has
+    left is reported as PeerLost before this rank launches any exchange, instead of surfacing
+    inside a collective.  Without it, a short process-group timeout is the bound.
     """
 
     def __init__(self, *, H, E, k, I, T_max, router_w=None, router_bias=None, local_w13=None, local_w2=None,
-                 shared_w13=None, shared_w2=None, group=None, backend=None, device=None):
+                 shared_w13=None, shared_w2=None, group=None, backend=None, device=None,
+                 liveness=None, liveness_timeout_s: float = 5.0):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -165,8 +181,41 @@ class ExpertParallelFfn:
             H=H, E=E, k=k, I=I, T_max=T_max, world=self.world, router_w=router_w, router_bias=router_bias,
             local_w13=local_w13, local_w2=local_w2, shared_w13=shared_w13, shared_w2=shared_w2, device=self.device)
         self.last_wire: WireBytes | None = None
+        self.liveness, self.liveness_timeout_s = liveness, liveness_timeout_s
+        self.step = 0
+
+    def _key(self, step: int, rank: int) -> str:
+        return f"afd_ep/{step}/{rank}"
+
+    def check_peers(self) -> None:
+        """Host-side check that every rank reached this step (no-op without a liveness store)."""
+        st = self.liveness
+        if st is None:
+            return
+        step = self.step
+        st.set(self._key(step, self.rank), "1")
+        keys = [self._key(step, r) for r in range(self.world)]
+        try:
+            st.wait(keys, datetime.timedelta(seconds=self.liveness_timeout_s))
+        except Exception as e:
+            missing = []
+            for r in range(self.world):
+                try:
+                    if not st.check([self._key(step, r)]):
+                        missing.append(r)
+                except Exception:
+                    missing.append(r)
+            raise PeerLost(step, missing or list(range(self.world))) from e
+        if step >= 2:
+            # every rank has set its key for step - 1, so all are done waiting on step - 2
+            try:
+                st.delete_key(self._key(step - 2, self.rank))
+            except Exception:
+                pass
+        self.step = step + 1
 
     def forward(self, hidden: torch.Tensor) -> torch.Tensor:
+        self.check_peers()
         T, H, k = hidden.shape[0], self.H, self.k
         b, g = self.backend, self.group
         idx, w = b.route(hidden, T)

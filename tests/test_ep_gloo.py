@@ -115,43 +115,124 @@ def test_block_tables_interleave_sources_per_expert():
     assert per_expert.tolist() == [2, 2]
 
 
-def _leaving_worker(rank, world, port, q):
-    """Rank 1 leaves between steps (after the group is up, before the next forward); rank 0's
-    next forward must end with an error from the group's short timeout, not hang."""
+class _CountingBackend:
+    """OracleRowsBackend that counts the steps that reached routing."""
+
+    def __init__(self, inner):
+        self.inner, self.routed = inner, 0
+
+    def route(self, hidden, T):
+        self.routed += 1
+        return self.inner.route(hidden, T)
+
+    def __getattr__(self, name):
+        return getattr(self.inner, name)
+
+
+def _leaving_worker(rank, world, port, q, use_store):
+    """Both ranks take one step; then rank 1 leaves (between steps) and rank 0 takes the next.
+    With a liveness store rank 0 must report PeerLost before it starts any exchange; without one,
+    its step must still end (an error from the exchange, or the process ending) rather than hang."""
     import datetime
     import time
+    from ep_support import OracleRowsBackend
+    from ffn_side_expert_b200.ep import PeerLost
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    store = None
+    if use_store:
+        store = dist.TCPStore("127.0.0.1", port + 1, world, is_master=(rank == 0),
+                              timeout=datetime.timedelta(seconds=20))
+    Wr, experts = _weights()
+    el = E // world
+    backend = _CountingBackend(OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K,
+                                                 local_experts=experts[rank * el:(rank + 1) * el], shared=experts[E]))
+    ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend, liveness=store, liveness_timeout_s=2.0)
+    hidden = torch.from_numpy(np.random.default_rng(3 + rank).normal(0, 1, (6, H)))
+    ep.forward(hidden)                                # step 0: everyone is here
     dist.barrier()
     if rank == 1:
-        os._exit(0)                                   # leaves without taking the next step
-    from ep_support import OracleRowsBackend
-    Wr, experts = _weights()
-    backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[:E // world], shared=experts[E])
-    ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
-    hidden = torch.from_numpy(np.random.default_rng(3).normal(0, 1, (6, H)))
+        os._exit(0)                                   # leaves between steps
     t0 = time.monotonic()
     try:
         ep.forward(hidden)
-        q.put(("no error", time.monotonic() - t0))
+        outcome = "no error"
+    except PeerLost as e:
+        outcome = f"PeerLost {e.missing}"
     except Exception as e:                            # the exchange reports the missing peer
-        q.put((type(e).__name__, time.monotonic() - t0))
+        outcome = type(e).__name__
+    q.put((outcome, time.monotonic() - t0, backend.routed))
+    q.close()
+    q.join_thread()                                   # flush the result before leaving without teardown
     os._exit(0)
 
 
-def test_a_rank_that_leaves_ends_the_others_step_with_an_error():
+def _run_leaving(use_store, port):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 27600 + os.getpid() % 1000
-    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, q, use_store)) for r in range(2)]
     for p in procs:
         p.start()
+    procs[0].join(90)
+    still = procs[0].is_alive()
+    for p in procs:
+        if p.is_alive():
+            p.kill()                                  # this test's own child, by handle
+        p.join(10)
+    assert not still, "rank 0 did not finish its step"
+    return None if q.empty() else q.get(timeout=5), procs[0].exitcode
+
+
+def test_a_rank_that_leaves_is_found_on_the_host_before_the_exchange():
+    got, code = _run_leaving(True, 25600 + 2 * (os.getpid() % 500))
+    assert code == 0 and got is not None
+    outcome, seconds, routed = got
+    assert outcome == "PeerLost [1]"
+    assert routed == 1                                # the second step stopped before routing
+    assert seconds < 10.0
+
+
+def test_without_a_store_the_step_still_ends():
+    got, code = _run_leaving(False, 24600 + 2 * (os.getpid() % 500))
+    # gloo reports a vanished peer as an error, or (from its own threads) ends the process
+    assert (got is not None and got[0] != "no error") or code != 0, (got, code)
+
+
+def _steps_worker(rank, world, port, q):
+    import datetime
+    from ep_support import OracleRowsBackend
+    from oracle import moe
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=20))
     try:
-        outcome, seconds = q.get(timeout=90)
+        store = dist.TCPStore("127.0.0.1", port + 1, world, is_master=(rank == 0),
+                              timeout=datetime.timedelta(seconds=20))
+        Wr, experts = _weights()
+        el = E // world
+        backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[rank * el:(rank + 1) * el],
+                                    shared=experts[E])
+        ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend, liveness=store)
+        worst = 0.0
+        for step in range(4):
+            hidden = torch.from_numpy(np.random.default_rng(50 + 10 * step + rank).normal(0, 1, (5 + step, H)))
+            out = ep.forward(hidden)
+            ref = moe.forward(hidden.numpy(), Wr, None, lambda e: {"w13": experts[e][0], "w2": experts[e][1]},
+                              E, K, 1)["out"]
+            worst = max(worst, float(np.max(np.abs(out.numpy() - ref))))
+        q.put((rank, worst, ep.step))
     finally:
-        for p in procs:
-            p.join(30)
-            if p.is_alive():
-                p.kill()                              # this test's own child, by handle
-    assert outcome != "no error"
-    assert seconds < 60
+        dist.destroy_process_group()
+
+
+def test_liveness_checked_steps_match_the_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 23600 + 2 * (os.getpid() % 500)
+    procs = [ctx.Process(target=_steps_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    for rank, worst, steps in sorted(q.get(timeout=10) for _ in range(2)):
+        assert worst <= 1e-12 and steps == 4, (rank, worst, steps)
