@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
 # of the decode shape, from a one-pass ncu capture of two launches at T=256, H=7168, E=256,
-# k=8, I=2048 with the shared expert (profiles/expert_ffn_fused_dsv3_256.md): 23 076 790 784 and
+# k=8, I=2048 with the shared expert: 23 076 790 784 and
 # 23 081 380 864 bytes for 257 touched experts.  Traffic grows with the experts whose weights
 # are streamed, and it is reported only while the kernel source and its instantiation are the
 # ones that were captured.

@@ -12,10 +12,16 @@ Where these roundings decide a stored code, the decision is taken in fp32 -- the
 of the GPU kernel: the scale is an fp32 quotient and each element is the fp32 quotient
 x / scale before it is rounded to e4m3.
 
-Pins (tests/test_oracle_fp8.py): every one of the 256 codes decodes to the value printed in
-tests/golden/e4m3_codes.txt and re-encodes to itself; exact midpoints round to the even
-code; values past 448 saturate; random fp32 values match an independent library routine
-(ml_dtypes.float8_e4m3fn) wherever that routine is in range.
+Pins (tests/test_oracle_fp8.py): every one of the 256 codes decodes to the value two
+independent implementations give (ml_dtypes.float8_e4m3fn and torch.float8_e4m3fn) and
+re-encodes to itself; a few codes are checked by hand (1, 448, the smallest normal and
+subnormal, -2, NaN); exact midpoints round to the even code; values past 448 saturate;
+random fp32 values match ml_dtypes wherever it is in range.  quantize_rows is checked against
+torch's own fp32 quotients and e4m3 conversion, and on rows whose fp32 quotient lands exactly
+on a rounding midpoint, so that an fp64 scale would give a different code.  The quantisation
+points of the W8A8 layer (hidden row, SwiGLU row) are pinned by a hand-worked expert and a
+scalar-loop layer (tests/test_oracle_expert.py::test_w8a8_worked_example and
+::test_w8a8_forward_against_scalar_loops).
 """
 from __future__ import annotations
 

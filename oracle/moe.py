@@ -12,7 +12,7 @@ What the pages fix (cited by page title and section):
   experts, each expert is a large matrix multiplication, and the expert outputs are combined
   back per token (A/F 分离, 为什么要拆 and 机制).
 
-What the pages leave open, and the reading taken here (each one listed in the design doc):
+What the pages leave open, and the reading taken here:
 - router: logits l = hidden . Wr^T (+ bias), in fp32 on the device, fp64 here; the hidden
   state enters as the bf16 values the device receives.
 - selection: the k largest logits, in descending order, ties to the lower expert index.

@@ -82,3 +82,49 @@ def test_quantize_rows_properties():
     deq = q * s[:, None].astype(np.float64)
     err = np.abs(deq - x)
     assert np.all(err <= np.maximum(np.abs(x) * 2.0 ** -4, s[:, None] * 2.0 ** -10) + 1e-12)
+
+
+def _torch_fp32_quantize(x32):
+    """The same per-row quantisation evaluated by torch: fp32 amax, fp32 quotient amax / 448,
+    fp32 quotient x / scale, then torch's own float8_e4m3fn conversion (round to nearest even)."""
+    x = torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32))
+    amax = x.abs().amax(dim=1)
+    s = torch.where(amax > 0, amax / torch.tensor(448.0, dtype=torch.float32), torch.ones_like(amax))
+    q = (x / s[:, None]).to(torch.float8_e4m3fn).to(torch.float64)
+    return q.numpy(), s.numpy()
+
+
+def test_quantize_rows_matches_torch_fp32_path():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((64, 257)) * rng.choice([1e-4, 1e-2, 1.0, 50.0, 3e4], (64, 1))).astype(np.float32)
+    x[5] = 0.0                                          # zero row: scale 1, codes 0
+    x[9] = 0.0
+    x[9, 100] = -3.0                                    # one non-zero: it maps to -448
+    q, s = fp8.quantize_rows(x)
+    qt, st = _torch_fp32_quantize(x)
+    assert np.array_equal(s, st)
+    assert np.array_equal(q, qt)
+
+
+# Rows whose fp32 quotient x / scale lands exactly on an e4m3 rounding midpoint, so that the
+# precision of the scale decides the code (the W8A8 reading: scale and quotient are fp32):
+#   amax = 0x1.143802p-1, scale = fp32(amax / 448) = 0x1.3badbap-10 (above the exact quotient),
+#   x = 0x1.4f6896p-6: fp32(x / scale) = 17.0 exactly, the midpoint of 16 and 18; ties to even
+#   give 16.  With an fp64 scale and quotient, x / (amax / 448) = 17.000000994..., which gives 18.
+#   amax = 0x1.9e97e4p+2, x = 0x1.f76f4ep-1: fp32(x / scale) = 68.0 exactly, the midpoint of 64
+#   and 72 -> 64 (an fp64 scale gives 68.0000047... -> 72).
+FP32_TIE_ROWS = [
+    (float.fromhex("0x1.143802p-1"), float.fromhex("0x1.4f6896p-6"), 16.0),
+    (float.fromhex("0x1.9e97e4p+2"), float.fromhex("0x1.f76f4ep-1"), 64.0),
+]
+
+
+def test_quantize_rows_scale_and_quotient_are_fp32():
+    x = np.array([[a, v] for a, v, _ in FP32_TIE_ROWS], dtype=np.float32)
+    q, s = fp8.quantize_rows(x)
+    assert s[0] == np.float32(float.fromhex("0x1.3badbap-10"))
+    for r, (_, _, code) in enumerate(FP32_TIE_ROWS):
+        assert q[r, 0] == 448.0
+        assert q[r, 1] == code
+    qt, st = _torch_fp32_quantize(x)
+    assert np.array_equal(q, qt) and np.array_equal(s, st)
