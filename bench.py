@@ -1,11 +1,14 @@
 """Benchmark of the FFN-service MoE layer on B200: tokens/s per layer and roofline fraction.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3_256] [--impl ours|reference]
+                    [--shapes dsv3_4096,w8a8_8192]
 
 One step = one afd_ffn_forward over one micro-batch (router, top-k, dispatch, gate/up GEMM
 with SwiGLU, down GEMM, shared expert, combine).  Default workload: the DeepSeek-V3 shaped
 decode micro-batch (T=256, H=7168, E=256 + 1 shared, top-8, I=2048, bf16) on seeded
-synthetic inputs.  Its 22.6 GB of expert weights are far larger than the 126 MB L2, so no
+synthetic inputs.  On one GPU the same line also carries, under "shapes", the T=4096
+Zipf-skewed bf16 micro-batch and the T=8192 W8A8 chunk, each timed the same way (K steps
+after W warm-ups) with its own roofline, stage split and clock record.  Its 22.6 GB of expert weights are far larger than the 126 MB L2, so no
 flush is needed between steps.  N > 1 runs one independent replica per GPU (the layer is
 not sharded: no collective on the data path); value = total tokens of all ranks / the
 slowest rank's time.  --impl reference times the fp64 CPU oracle on a bounded sample of the
@@ -80,7 +83,7 @@ def algorithmic(cfg, counts) -> dict:
     # the fused bf16 expert kernel (gate/up + SwiGLU + down): weights, dispatched rows in, outputs out
     expert = w13 + w2 + rows * H * b + rows * H * 4
     flops = 6 * H * I * (T * k + S * T) + 2 * T * H * E
-    return {"weight_bytes": w13 + w2, "act_bytes": act, "flops": flops, "gemm13_bytes": gemm13,
+    return {"weight_bytes": w13 + w2, "w13_bytes": w13, "act_bytes": act, "flops": flops, "gemm13_bytes": gemm13,
             "expert_bytes": expert,
             "gemm13_flops": 4 * H * I * rows, "touched_experts": n}
 
@@ -114,7 +117,7 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -129,7 +132,7 @@ class ClockSampler:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         time.sleep(0.3)
@@ -221,18 +224,14 @@ def workload_label(args) -> str:
     return args.config + (f"[{','.join(over)}]" if over else "")
 
 
-def run_ours(args, rank, world, local_rank):
+def time_forward(layer, h, out, cfg, args, world, local_rank) -> dict:
+    """W warm-up forwards, then K timed forwards back to back with CUDA events around the
+    whole region and around the dominant kernel (stage 5 -> 6: the fused expert kernel of the
+    bf16 decode shape, else the gate/up GEMM), nvidia-smi clocks sampled meanwhile; then a
+    second pass of K forwards with every stage boundary recorded for the per-stage split."""
     import ffn_side_expert_b200 as afd
-    cfg = workload(args)
-    torch.cuda.set_device(local_rank)
-    device = torch.device("cuda", local_rank)
-    hidden, Wr, bias, dev = build_inputs(cfg, device)
-    layer = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S,
-                       fp8=cfg.dtype == "fp8", weights=dev)
-    h = hidden.to(device)
-    out = torch.empty_like(h)
+    device = h.device
     stream = torch.cuda.current_stream()
-
     for _ in range(args.warmup):
         layer.forward(h, out)
     torch.cuda.synchronize()
@@ -247,9 +246,6 @@ def run_ours(args, rank, world, local_rank):
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=cfg.E)
     acct = algorithmic(cfg, counts)
 
-    # per-step events on the launch stream.  Timed region: only the two around the dominant
-    # kernel (stage 5: the fused expert kernel, or the gate/up GEMM); a second pass records
-    # every stage boundary for the per-stage breakdown.
     nev = afd.AFD_FFN_NUM_STAGES + 1
     K0, K1 = 5, 6
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
@@ -259,7 +255,6 @@ def run_ours(args, rank, world, local_rank):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
 
-    # timed region: K forwards back to back, the dominant kernel bracketed by CUDA events
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
@@ -276,12 +271,30 @@ def run_ours(args, rank, world, local_rank):
     st = layer.get_error()
     if st != afd.AFD_OK:
         raise afd.AfdError(st, "timed region")
-    # per-stage breakdown: the same K forwards with every stage boundary recorded
     for i in range(args.steps):
         layer.set_stage_events(ev[i])
         layer.forward(h, out)
     torch.cuda.synchronize()
     layer.set_stage_events(None)
+    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(nev - 1)]
+                         for i in range(args.steps)]).mean(axis=0)
+    return {"ms": allreduce_max(ms, world), "kernel_ms": allreduce_max(kernel_ms, world),
+            "stage_ms": stage_ms, "acct": acct, "cfg": cfg, "clocks": clk.summary()}
+
+
+def run_ours(args, rank, world, local_rank):
+    import ffn_side_expert_b200 as afd
+    cfg = workload(args)
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    hidden, Wr, bias, dev = build_inputs(cfg, device)
+    layer = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S,
+                       fp8=cfg.dtype == "fp8", weights=dev)
+    h = hidden.to(device)
+    out = torch.empty_like(h)
+    stream = torch.cuda.current_stream()
+    res = time_forward(layer, h, out, cfg, args, world, local_rank)
+
     # the same K forwards without any events, timed the same way
     barrier(world)
     torch.cuda.synchronize()
@@ -294,8 +307,6 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier(world)
     plain_ms = u0.elapsed_time(u1) / args.steps
-    stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(nev - 1)]
-                         for i in range(args.steps)]).mean(axis=0)
 
     # the same forward replayed from a CUDA graph (launch gaps removed), timed the same way
     graph_ms = None
@@ -342,17 +353,34 @@ def run_ours(args, rank, world, local_rank):
         layer.forward_host(seq_in[i], seq_out[i])
     e2e_sync_s = (time.perf_counter() - t0) / args.steps
 
-    ms_max = allreduce_max(ms, world)
-    graph_max = allreduce_max(graph_ms, world)
-    plain_max = allreduce_max(plain_ms, world)
-    e2e_max = allreduce_max(e2e_s, world)
-    e2e_sync_max = allreduce_max(e2e_sync_s, world)
-    res = {"ms": ms_max, "kernel_ms": allreduce_max(kernel_ms, world), "graph_ms": graph_max, "plain_ms": plain_max, "e2e_s": e2e_max, "e2e_sync_s": e2e_sync_max, "stage_ms": stage_ms, "acct": acct, "cfg": cfg,
-           "clocks": clk.summary(), "bytes_io": hidden.numel() * 2}
+    res.update(graph_ms=allreduce_max(graph_ms, world), plain_ms=allreduce_max(plain_ms, world),
+               e2e_s=allreduce_max(e2e_s, world), e2e_sync_s=allreduce_max(e2e_sync_s, world),
+               bytes_io=hidden.numel() * 2)
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu"] = cpu_baseline(cfg, hidden, Wr, bias)
     layer.close()
+    del layer, dev, h, out, hin, hout, seq_in, seq_out
+    torch.cuda.empty_cache()
     return res
+
+
+def run_shape(name, args, world, local_rank) -> dict:
+    """One more workload timed like the headline (warm-up, K timed forwards, stage pass); its
+    handle and weights are freed before returning."""
+    import ffn_side_expert_b200 as afd
+    cfg = synth.CONFIGS[name]
+    device = torch.device("cuda", local_rank)
+    hidden, _, _, dev = build_inputs(cfg, device)
+    layer = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S,
+                       fp8=cfg.dtype == "fp8", weights=dev)
+    h = hidden.to(device)
+    out = torch.empty_like(h)
+    try:
+        return time_forward(layer, h, out, cfg, args, world, local_rank)
+    finally:
+        layer.close()
+        del layer, dev, h, out
+        torch.cuda.empty_cache()
 
 
 def barrier(world):
@@ -375,38 +403,97 @@ def job_throughput(tokens_per_replica: int, world: int, slowest_ms: float) -> fl
     return world * tokens_per_replica / (slowest_ms / 1e3)
 
 
-def report_ours(args, world, r) -> dict:
-    import ffn_side_expert_b200 as afd
-    cfg, acct = r["cfg"], r["acct"]
+def fused_decode(cfg) -> bool:
+    """The bf16 decode shape runs its expert GEMMs as one fused launch."""
+    return cfg.dtype == "bf16" and cfg.T * cfg.k <= 32 * cfg.E
+
+
+def launches_per_step(cfg) -> int:
+    """Library kernel launches of one forward: router GEMM, selection (top-k + refined weights),
+    dispatch count, dispatch scan, gather, schedule, then the fused expert kernel (bf16 decode
+    shape) or gate/up GEMM (+ W8A8 activation quantisation) and down GEMM, then combine; from
+    T = 2048 selection and refinement are two launches."""
+    n = 8 if fused_decode(cfg) else (10 if cfg.dtype == "fp8" else 9)
+    return n + (1 if cfg.T >= 2048 else 0)
+
+
+def rooflines(cfg, acct, ms, kernel_ms, traffic=None):
+    """(roofline of the dominant kernel, roofline of the whole path) for one workload.
+
+    Dominant kernel: the fused expert kernel of the bf16 decode shape, else the gate/up GEMM.
+    Its algorithmic bytes are the expert weights it must stream (touched experts only, plus
+    the e4m3 scales); its algorithmic FLOPs are 2 per multiply-add of its products.  It is
+    reported against whichever of the HBM and tensor-core peaks bounds it (the larger of
+    bytes / HBM and FLOPs / tensor peak), with the other fraction beside it.
+    Path: t_roof = max(FLOPs / tensor peak, (weight + activation bytes) / HBM) over t_step."""
     peaks, kind = load_peaks()
-    ms = r["ms"]
-    value = job_throughput(cfg.T, world, ms)
-    stage = dict(zip(afd.STAGE_NAMES, [float(x) for x in r["stage_ms"]]))
     hbm = peaks["hbm_gbs"]
-    if cfg.dtype == "bf16" and cfg.T * cfg.k <= 32 * cfg.E:  # decode shape: one fused launch
-        kname, kbytes = "expert FFN kernel (gate/up + SwiGLU + down, fused)", acct["expert_bytes"]
-        k_ms = r["kernel_ms"]  # stage 5 -> 6 of the timed region: the fused kernel
-        traffic = fused_traffic(cfg, acct)
+    mult = 2.0 if cfg.dtype == "fp8" else 1.0          # e4m3 vs bf16 dense tensor rate
+    tc = peaks["bf16_tflops"] * mult
+    tc_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * mult
+    if fused_decode(cfg):
+        kname, kbytes, kflops = ("expert FFN kernel (gate/up + SwiGLU + down, fused)", acct["weight_bytes"],
+                                 acct["flops"] - 2 * cfg.T * cfg.H * cfg.E)
     else:
-        kname, kbytes = "grouped_gemm gate/up + SwiGLU", acct["gemm13_bytes"]
-        k_ms = r["kernel_ms"]  # stage 5 -> 6 of the timed region: the gate/up GEMM
-        traffic = None
-    achieved = kbytes / (k_ms / 1e3) / 1e9
+        kname, kbytes, kflops = "grouped_gemm gate/up + SwiGLU", acct["w13_bytes"], acct["gemm13_flops"]
+    sec = kernel_ms / 1e3
+    gbs, tfs = kbytes / sec / 1e9, kflops / sec / 1e12
+    tensor_bound = kflops / (tc * 1e12) > kbytes / (hbm * 1e9)
+    roof = {"bound": "tensor" if tensor_bound else "hbm",
+            "kernel": kname,
+            "achieved": round(tfs if tensor_bound else gbs, 1),
+            "peak": tc if tensor_bound else hbm,
+            "unit": "TFLOP/s" if tensor_bound else "GB/s",
+            "frac": round((tfs / tc) if tensor_bound else (gbs / hbm), 4),
+            "traffic": traffic,
+            "peak_source": f"{kind} " + ("bf16_tflops x 2 (e4m3)" if tensor_bound and mult == 2 else
+                                         "bf16_tflops" if tensor_bound else "hbm_gbs"),
+            "algorithmic_bytes_per_launch": kbytes, "algorithmic_flops_per_launch": kflops,
+            "avg_launch_ms": round(kernel_ms, 4),
+            "hbm_frac": round(gbs / hbm, 4), "tensor_frac": round(tfs / tc, 4),
+            "tensor_frac_sustained": round(tfs / tc_sus, 4)}
     t_hbm = (acct["weight_bytes"] + acct["act_bytes"]) / (hbm * 1e9)
-    tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.dtype == "fp8" else 1.0)
-    t_tc = acct["flops"] / (tc_peak * 1e12)
+    t_tc = acct["flops"] / (tc * 1e12)
     t_roof = max(t_hbm, t_tc)
     # the same bound with the tensor peak a GEMM sustains under the power cap (the timed steps
     # run back to back, and the clock record shows sw_power_cap under load)
-    tc_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (2.0 if cfg.dtype == "fp8" else 1.0)
     t_roof_sus = max(t_hbm, acct["flops"] / (tc_sus * 1e12))
-    # router GEMM, selection (top-k + refined weights), dispatch count, dispatch scan, gather,
-    # schedule, then the fused expert kernel (bf16 decode shape) or gate/up GEMM (+ W8A8
-    # activation quantisation) and down GEMM, then combine
-    fused = cfg.dtype == "bf16" and cfg.T * cfg.k <= 32 * cfg.E
-    launches = 8 if fused else (10 if cfg.dtype == "fp8" else 9)
-    if cfg.T >= 2048:  # selection and refinement as two launches
-        launches += 1
+    path = {"t_roof_ms": round(t_roof * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
+            "t_tensor_ms": round(t_tc * 1e3, 4), "frac": round(t_roof * 1e3 / ms, 4),
+            "weight_bytes": acct["weight_bytes"], "act_bytes": acct["act_bytes"],
+            "flops": acct["flops"], "touched_experts": acct["touched_experts"],
+            "peaks": f"{kind}: hbm {hbm} GB/s, tensor {tc} TFLOP/s (burst)",
+            "frac_sustained": round(t_roof_sus * 1e3 / ms, 4),
+            "t_roof_sustained_ms": round(t_roof_sus * 1e3, 4),
+            "peaks_sustained": f"{kind}: hbm {hbm} GB/s, tensor {round(tc_sus, 1)} TFLOP/s (sustained)"}
+    return roof, path
+
+
+def report_shape(args, world, r) -> dict:
+    """The JSON object of one extra workload (same timing as the headline's value)."""
+    import ffn_side_expert_b200 as afd
+    cfg = r["cfg"]
+    roof, path = rooflines(cfg, r["acct"], r["ms"], r["kernel_ms"])
+    return {"value": round(job_throughput(cfg.T, world, r["ms"]), 1), "unit": "tokens/s",
+            "ms_per_step": round(r["ms"], 4),
+            "dtype": "fp8_e4m3" if cfg.dtype == "fp8" else "bf16",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+                       "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed,
+                       "routing": "Zipf-skewed (router bias)" if cfg.has_bias else "uniform"},
+            "roofline": roof, "path_roofline": path,
+            "stage_ms": {k: round(float(v), 4) for k, v in zip(afd.STAGE_NAMES, r["stage_ms"])},
+            "gpu_launches": launches_per_step(cfg) * args.steps, "clocks": r["clocks"]}
+
+
+def report_ours(args, world, r) -> dict:
+    import ffn_side_expert_b200 as afd
+    cfg, acct = r["cfg"], r["acct"]
+    ms = r["ms"]
+    value = job_throughput(cfg.T, world, ms)
+    stage = dict(zip(afd.STAGE_NAMES, [float(x) for x in r["stage_ms"]]))
+    traffic = fused_traffic(cfg, acct) if fused_decode(cfg) else None
+    roof, path = rooflines(cfg, acct, ms, r["kernel_ms"], traffic)
+    launches = launches_per_step(cfg)
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
@@ -415,21 +502,9 @@ def report_ours(args, world, r) -> dict:
         "config": {"workload": workload_label(args), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
                    "I": cfg.I, "n_shared": cfg.S, "weights": cfg.dtype, "seed": cfg.seed,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (expert weights 22.6 GB >> 126 MB)"},
-        "roofline": {"bound": "hbm", "kernel": kname,
-                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": traffic,
-                     "peak_source": f"{kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": kbytes,
-                     "avg_launch_ms": round(k_ms, 4)},
-        "path_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
-                          "t_tensor_ms": round(t_tc * 1e3, 4), "frac": round(t_roof * 1e3 / ms, 4),
-                          "weight_bytes": acct["weight_bytes"], "act_bytes": acct["act_bytes"],
-                          "flops": acct["flops"], "touched_experts": acct["touched_experts"],
-                          "peaks": f"{kind}: hbm {hbm} GB/s, tensor {tc_peak} TFLOP/s (burst)",
-                          "frac_sustained": round(t_roof_sus * 1e3 / ms, 4),
-                          "t_roof_sustained_ms": round(t_roof_sus * 1e3, 4),
-                          "peaks_sustained": f"{kind}: hbm {hbm} GB/s, tensor {round(tc_sus, 1)} TFLOP/s (sustained)"},
+                   "l2": f"inputs larger than L2 (expert weights {acct['weight_bytes'] / 1e9:.1f} GB >> 126 MB)"},
+        "roofline": roof,
+        "path_roofline": path,
         "stage_ms": {k: round(v, 4) for k, v in stage.items()},
         "uninstrumented": {"value": round(job_throughput(cfg.T, world, r["plain_ms"]), 1), "unit": "tokens/s",
                            "ms_per_step": round(r["plain_ms"], 4),
@@ -668,6 +743,8 @@ def main(argv=None):
                     help="profiling only: override the micro-batch size (a smaller case of the same kernels)")
     ap.add_argument("--E", type=int, default=None,
                     help="profiling only: override the number of routed experts")
+    ap.add_argument("--shapes", default="dsv3_4096,w8a8_8192",
+                    help="comma-separated workloads timed after the headline one (1 GPU only; '' for none)")
     ap.add_argument("--period", action="store_true",
                     help="measure the FFN-service micro-pipeline period with a host attention stub (1 GPU)")
     args = ap.parse_args(argv)
@@ -696,8 +773,18 @@ def main(argv=None):
                                              device_id=torch.device("cuda", local_rank))
     try:
         r = run_ours(args, rank, world, local_rank)
+        # the other shapes the metric names, timed the same way on the same GPU after the
+        # headline one (replica runs across GPUs time the headline workload only)
+        shapes = {}
+        names = [n for n in args.shapes.split(",") if n and n != args.config] if world == 1 else []
+        if args.T is None and args.E is None:
+            for name in names:
+                shapes[name] = report_shape(args, world, run_shape(name, args, world, local_rank))
         if rank == 0:
-            print(json.dumps(report_ours(args, world, r)), flush=True)
+            line = report_ours(args, world, r)
+            if shapes:
+                line["shapes"] = shapes
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

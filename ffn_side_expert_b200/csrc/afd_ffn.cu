@@ -50,6 +50,7 @@ struct afd_ffn_handle {
   int device = 0;
   int num_sms = 0;
   int pair_grid = 0;  // CTAs of the CTA-pair GEMMs: 2 x the pairs that fit on the device at once
+  int fused_grid = 0; // CTAs of the fused decode launch (cooperative: all resident at once)
   bool fp8 = false;
   int G = 0;       // E + n_shared
   int R_max = 0;   // rows of the dispatched-row buffers: T_max * (k + 1)
@@ -91,6 +92,7 @@ struct afd_ffn_handle {
   // bf16 large micro-batches: f16 copy of W2 and the f16 activation plane (single-term down GEMM)
   void* w2h = nullptr;       // [E+S][H][I] f16, owned; NULL when unused
   bool act16 = false;
+  float f16_bound = 0.f;     // 2 C / 32768 (w13_norm_bound_kernel): the f16 act row scales' input
   CUtensorMap tm_w2h, tm_act16;
   CUtensorMap tm_xp[2], tm_act[2];  // token rows for the [narrow, wide] shapes (box heights differ)
   cudaStream_t last_stream = nullptr;
@@ -374,9 +376,50 @@ void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const Gem
     cfg.numAttrs = 1;
     cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>, a, b, a2 ? *a2 : a, b2 ? *b2 : b,
                        args);
+  } else if constexpr (MODE == 3) {
+    // the fused kernel's down units wait for act tiles that other CTAs produce, so every CTA of
+    // the grid must be resident at once: a cooperative launch guarantees it, or fails (with a
+    // launch error that the stage's cudaGetLastError check returns) when it cannot be met
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = gemm_smem_bytes<BN, ST, SPLIT, MODE>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, false, ACT16>, a, b, a2 ? *a2 : a,
+                       b2 ? *b2 : b, args);
   } else {
     grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, false, ACT16>
         <<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
+  }
+}
+
+// CTAs of the fused (MODE 3) launch: one per SM when that many fit at once (the kernel holds
+// one CTA per SM by its shared memory), else as many as can be co-resident; 0 when the device
+// cannot launch it cooperatively.
+template <bool FP8>
+int fused_grid(int num_sms, int device) {
+  using P = GemmPair<FP8, kNarrow>;
+  if constexpr (!P::fused) {
+    return num_sms;
+  } else {
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device) != cudaSuccess || !coop) {
+      cudaGetLastError();
+      return 0;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_gemm_kernel<P::bn1, P::stf, FP8, 3, true>,
+                                                      kGemmThreads, gemm_smem_bytes<P::bn1, P::stf, true, 3>()) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return std::min(num_sms, per_sm * num_sms);
   }
 }
 
@@ -496,7 +539,7 @@ int run_permute(afd_ffn_handle* h, const void* hidden, const int32_t* idx, int T
                                                h->xp, h->xscale);
   else
     gather_rows_kernel<false><<<T, 256, 0, s>>>(hb, idx, h->chunk_base, pos, src, T, c.k, c.E, c.H, c.n_shared,
-                                                h->xp, h->xscale);
+                                                h->xp, h->xscale, h->act16 ? h->f16_bound : 0.f);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -540,7 +583,7 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
     f.out_ld2 = c.H;
     f.mt1 = c.I / 128;
     record(h, 5, s);
-    launch_gemm<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>(h->num_sms, h->tm_w13, h->tm_xp[shape], f, s,
+    launch_gemm<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>(h->fused_grid, h->tm_w13, h->tm_xp[shape], f, s,
                                                                 &h->tm_w2, &h->tm_act[shape]);
     record(h, 6, s);
     record(h, 7, s);
@@ -815,12 +858,28 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
     if (!h->act16) {
       cudaFree(h->w2h);
       h->w2h = nullptr;
+    } else {
+      // bound of the SwiGLU output per unit of ||x||^2, for the f16 row scales
+      unsigned* c_bits = reinterpret_cast<unsigned*>(h->err) + 1;
+      w13_norm_bound_kernel<<<4 * h->num_sms, 256>>>(static_cast<const __nv_bfloat16*>(weights->w13),
+                                                     static_cast<int>(G), c.I, c.H, c_bits);
+      unsigned bits = 0;
+      e = cudaGetLastError();
+      if (e == cudaSuccess) e = cudaMemcpy(&bits, c_bits, sizeof(unsigned), cudaMemcpyDeviceToHost);
+      if (e == cudaSuccess) e = cudaMemset(c_bits, 0, sizeof(unsigned));
+      if (e != cudaSuccess) { cudaFree(h->w2h); cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+      float C = 0.f;
+      std::memcpy(&C, &bits, sizeof(float));
+      // a zero (or NaN) bound still gives every row the scale 1
+      h->f16_bound = std::max(2.0f * C / 32768.0f, 1e-30f);
     }
   }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
-  if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }
+  if (e != cudaSuccess) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return cuda_fail(nullptr, e); }
   h->pair_grid = h->fp8 ? pair_grid<true>(h->num_sms) : pair_grid<false>(h->num_sms);
-  if (h->pair_grid < 2) { cudaFree(h->ws); delete h; return AFD_ERR_UNSUPPORTED; }
+  if (h->pair_grid < 2) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return AFD_ERR_UNSUPPORTED; }
+  h->fused_grid = h->fp8 ? fused_grid<true>(h->num_sms, dev) : fused_grid<false>(h->num_sms, dev);
+  if (h->fused_grid < 1) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return AFD_ERR_UNSUPPORTED; }
   router_split_planes_kernel<<<256, 256>>>(weights->router_w, static_cast<size_t>(c.E) * c.H,
                                            static_cast<__nv_bfloat16*>(h->wr_planes));
   e = cudaGetLastError();
@@ -1136,6 +1195,9 @@ extern "C" int afd_ffn_expert_rows(afd_ffn_handle* h, const void* rows, const in
   h->last_stream = s;
   const size_t H = c.H;
   AFD_CUDA(h, cudaMemcpyAsync(h->xp, rows, static_cast<size_t>(n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
+  if (h->act16 && !use_narrow(h, n_rows))  // the f16 activations' row scales
+    f16_row_scale_kernel<<<n_rows, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->xp), c.H, h->f16_bound,
+                                                h->xscale);
   // group offsets from the per-expert counts (one "chunk")
   dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(counts, 1, c.E, h->counts, h->offsets, h->chunk_base);
   AFD_CUDA(h, cudaGetLastError());

@@ -118,6 +118,59 @@ __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half
   if (big) atomicOr(overflow, 1);
 }
 
+// Weight side of the f16 row scale: for every expert g and intermediate column i,
+// |silu(x.wg_i) (x.wu_i)| <= |x.wg_i| |x.wu_i| <= ||x||^2 ||wg_i|| ||wu_i||  (|silu(z)| <= |z|;
+// Cauchy-Schwarz), so C = max over g, i of ||wg_i|| ||wu_i|| bounds every act value of a token
+// row by ||x||^2 C.  Warps stride over the (g, i) pairs of w13 [G][2I][H] bf16; *c_bits receives
+// C as the bits of a non-negative float (atomicMax on the bits orders non-negative floats).
+__global__ void __launch_bounds__(256)
+w13_norm_bound_kernel(const __nv_bfloat16* __restrict__ w13, int G, int I, int H, unsigned* c_bits) {
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  float c = 0.f;
+  for (long long p = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       p < static_cast<long long>(G) * I; p += nwarps) {
+    const long long g = p / I, i = p - g * I;
+    const uint4* rg = reinterpret_cast<const uint4*>(w13 + (g * 2 * I + i) * H);
+    const uint4* ru = reinterpret_cast<const uint4*>(w13 + (g * 2 * I + I + i) * H);
+    float sg = 0.f, su = 0.f;
+    for (int v = lane; v < H / 8; v += 32) {
+      const uint4 a = rg[v], b = ru[v];
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 fa = __bfloat1622float2(pa[j]), fb = __bfloat1622float2(pb[j]);
+        sg = fmaf(fa.x, fa.x, fmaf(fa.y, fa.y, sg));
+        su = fmaf(fb.x, fb.x, fmaf(fb.y, fb.y, su));
+      }
+    }
+    sg = warp_sum(sg);
+    su = warp_sum(su);
+    c = fmaxf(c, sqrtf(sg) * sqrtf(su));
+  }
+  if (lane == 0) atomicMax(c_bits, __float_as_uint(c));
+}
+
+// f16 row scales of rows that arrive already dispatched (one CTA of 256 threads per row).
+__global__ void __launch_bounds__(256)
+f16_row_scale_kernel(const __nv_bfloat16* __restrict__ rows, int H, float f16_bound, float* __restrict__ xscale) {
+  __shared__ float red[32];
+  const uint4* r4 = reinterpret_cast<const uint4*>(rows + static_cast<size_t>(blockIdx.x) * H);
+  float ss = 0.f;
+  for (int v = threadIdx.x; v < H / 8; v += blockDim.x) {
+    const uint4 x = r4[v];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(b[j]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+  ss = block_sum(ss, red);
+  if (threadIdx.x == 0) xscale[blockIdx.x] = f16_row_scale(ss, f16_bound);
+}
+
 // Widen bf16 rows to fp32 (copy-out of the W8A8 expert outputs by afd_ffn_expert_gemm).
 __global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, size_t n) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;

@@ -116,15 +116,17 @@ dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int 
 // are written, and hidden row t is copied to every dispatched row and (shared expert) to row
 // T*k + t.  bf16 rows move as 16-byte vectors.  W8A8: the row is quantised first --
 // scale = amax / 448 (1 for a zero row), e4m3 = round-to-nearest-even, saturating, of the fp32
-// quotient x / scale -- and the scale travels with every copy.
+// quotient x / scale -- and the scale travels with every copy.  bf16 with f16_bound > 0 (the
+// f16 activations of large micro-batches): the row's power-of-two act scale (f16_row_scale of
+// ||x||^2) is written for every copy instead.
 template <bool FP8>
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __restrict__ idx,
                    const int32_t* __restrict__ chunk_base, int32_t* __restrict__ pos,
                    int32_t* __restrict__ src, int T, int k, int E, int H, int with_shared,
-                   uint8_t* __restrict__ xp, float* __restrict__ xscale) {
+                   uint8_t* __restrict__ xp, float* __restrict__ xscale, float f16_bound = 0.f) {
   __shared__ int dst[34];  // up to 32 routed + 1 shared destinations; count in [33]
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
   if (tid < 32) {
@@ -151,10 +153,24 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ hidden, const int32_t* __re
   const __nv_bfloat16* row = hidden + static_cast<size_t>(t) * H;
   const uint4* s4 = reinterpret_cast<const uint4*>(row);
   if constexpr (!FP8) {
+    const bool scaled = f16_bound > 0.f && xscale != nullptr;  // uniform over the CTA
+    float ss = 0.f;
     for (int v = tid; v < H / 8; v += blockDim.x) {
       const uint4 x = s4[v];
       for (int d = 0; d < nd; ++d)
         reinterpret_cast<uint4*>(xp + static_cast<size_t>(dst[d]) * H * 2)[v] = x;
+      if (scaled) {
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(b[i]);
+          ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+        }
+      }
+    }
+    if (scaled) {
+      ss = block_sum(ss, red);
+      if (tid < nd) xscale[dst[tid]] = f16_row_scale(ss, f16_bound);
     }
   } else {
     float amax = 0.f;

@@ -232,7 +232,9 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
 
 // ACT16 (bf16 large micro-batches): the gate/up epilogue stores the SwiGLU output as one f16
 // plane (MODE 0), and the down GEMM multiplies it by an f16 copy of W2 (MODE 1, kind::f16 with
-// f16 operands) -- f16 keeps 10 mantissa bits where bf16 keeps 7, so one term suffices.
+// f16 operands) -- f16 keeps 10 mantissa bits where bf16 keeps 7, so one term suffices.  Each
+// token row is stored divided by its power-of-two scale b_scale[row] (f16_row_scale: the row's
+// bound on |act| stays inside the f16 range), and the down epilogue multiplies it back.
 template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool PAIR = false, bool ACT16 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -508,9 +510,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           sa1 = __ldg(args.a_scale + static_cast<size_t>(w.g) * args.a_rows + wrow1);
         }
         for (int c = c_first; c < w.n16; c += kCStep) {
-          // W8A8: lane i < 16 fetches the scale of token c + i once; shuffled to all lanes below
+          // W8A8 (and the f16 activations): lane i < 16 fetches the scale of token row c + i once;
+          // shuffled to all lanes below
           float sb_lane = 0.f;
-          if constexpr (FP8) {
+          if constexpr (FP8 || ACT16) {
             if (lane < 16 && c + lane < w.rows) sb_lane = __ldg(args.b_scale + w.row0 + c + lane);
           }
           uint32_t r0[16], r1[16];
@@ -538,7 +541,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           for (int i = 0; i < 16; ++i) {
             const int n = c + i;
             float sb = 1.f;
-            if constexpr (FP8) sb = __shfl_sync(0xffffffffu, sb_lane, i);
+            if constexpr (FP8 || ACT16) sb = __shfl_sync(0xffffffffu, sb_lane, i);
             if (n < w.rows) {
               const size_t row = static_cast<size_t>(w.row0 + n);
               float v0 = __uint_as_float(r0[i]);
@@ -551,8 +554,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float act = silu_f(v0) * v1;  // gate tile first, up tile second
                 if constexpr (FP8) {
                   static_cast<float*>(args.out)[row * args.out_ld + wrow0] = act;
-                } else if constexpr (ACT16) {
-                  static_cast<__half*>(args.out)[row * args.out_ld + wrow0] = __float2half_rn(act);
+                } else if constexpr (ACT16) {  // act / s, s the row's power-of-two f16 scale (exact)
+                  static_cast<__half*>(args.out)[row * args.out_ld + wrow0] = __float2half_rn(act * __frcp_rn(sb));
                 } else {
                   const __nv_bfloat16 hi = __float2bfloat16_rn(act);
                   const __nv_bfloat16 lo = __float2bfloat16_rn(act - __bfloat162float(hi));
@@ -567,6 +570,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               } else {
                 float* y = static_cast<float*>(MODE == 3 ? args.out2 : args.out) +
                            row * (MODE == 3 ? args.out_ld2 : args.out_ld);
+                if constexpr (ACT16) {  // undo the row's f16 scale of the activations
+                  v0 *= sb;
+                  v1 *= sb;
+                }
                 y[wrow0] = v0;
                 if constexpr (S::kNDU == 2) y[wrow1] = v1;
               }

@@ -26,8 +26,8 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-from . import (AFD_OK, AfdError, AfdFfn, afd_ffn_combine_rows, afd_ffn_copy_row_blocks, afd_ffn_dispatch_rows,
-               afd_ffn_expert_rows, afd_ffn_route_static)
+from . import (AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS, AFD_OK, AfdError, AfdFfn, afd_ffn_combine_rows,
+               afd_ffn_copy_row_blocks, afd_ffn_dispatch_rows, afd_ffn_expert_rows, afd_ffn_route_static)
 
 
 def block_tables(recv_counts: torch.Tensor):
@@ -78,7 +78,8 @@ class PeerLost(RuntimeError):
 
     def __init__(self, step: int, missing: list):
         self.step, self.missing = step, missing
-        super().__init__(f"ranks {missing} did not reach step {step}")
+        super().__init__(f"ranks {missing} did not reach step {step}" if missing else
+                         f"step {step} was aborted by a rank whose wait for the others ran out")
 
 
 class CudaRowsBackend:
@@ -97,6 +98,7 @@ class CudaRowsBackend:
             self.shared = AfdFfn(T_max=T_max, H=H, E=1, k=1, I=I, n_shared=0, fp8=False,
                                  weights={"router_w": dummy_router[:1], "w13": shared_w13[None], "w2": shared_w2[None]})
         self.scratch = torch.empty(2 * ((T_max + 127) // 128) * E, dtype=torch.int32, device=device)
+        self.route_chunk = max(1, AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS // E)
         self.keep = [dummy_router]
 
     @staticmethod
@@ -107,8 +109,12 @@ class CudaRowsBackend:
     def route(self, hidden, T):
         idx = torch.empty((T, self.k), dtype=torch.int32, device=self.device)
         w = torch.empty((T, self.k), dtype=torch.float32, device=self.device)
-        self._ok(afd_ffn_route_static(hidden, self.router_w, self.router_bias, T, self.H, self.E, self.k, idx, w),
-                 "afd_ffn_route_static")
+        # the allocation-free router holds the partial logits of at most route_chunk tokens,
+        # so a larger micro-batch is routed in consecutive chunks on the same stream
+        for t0 in range(0, T, self.route_chunk):
+            n = min(self.route_chunk, T - t0)
+            self._ok(afd_ffn_route_static(hidden[t0:t0 + n], self.router_w, self.router_bias, n, self.H, self.E,
+                                          self.k, idx[t0:t0 + n], w[t0:t0 + n]), "afd_ffn_route_static")
         return idx, w
 
     def dispatch(self, hidden, idx, T):
@@ -158,11 +164,20 @@ class ExpertParallelFfn:
     Every rank calls forward() with its own micro-batch (the same T on all ranks is not
     required).  `backend` defaults to CudaRowsBackend built from the arguments.
 
+    T_max: the largest micro-batch a rank may pass; forward() refuses a larger one with
+    ValueError before any device work (the dispatch scratch and the expert handles are sized
+    for it).
+
     liveness: optional torch.distributed Store that every rank of the group reaches.  With it,
-    each forward first checks on the host that every rank has reached the same step (each
-    rank sets its key, then waits up to liveness_timeout_s for the others').  A rank that has
-    left is reported as PeerLost before this rank launches any exchange, instead of surfacing
-    inside a collective.  Without it, a short process-group timeout is the bound.
+    each forward first checks on the host that every rank has reached the same step: each
+    rank sets its arrival key, then waits up to liveness_timeout_s for the others'.  The step
+    is then decided once, atomically, in the store (compare_set of the step's state key): "go"
+    by the first rank that saw every arrival, or "abort" by the first rank whose wait ran out.
+    Every rank acts on the decided state, so either all of them run the exchange or all of
+    them raise PeerLost -- a rank that arrives after another gave up finds "abort" and raises
+    too, instead of entering a collective alone.  A rank that has left, or a store that can no
+    longer be reached, is reported as PeerLost before this rank launches any exchange.
+    Without a store, a short process-group timeout is the bound.
     """
 
     def __init__(self, *, H, E, k, I, T_max, router_w=None, router_bias=None, local_w13=None, local_w2=None,
@@ -174,6 +189,7 @@ class ExpertParallelFfn:
         if E % self.world:
             raise ValueError("E must split evenly over the ranks")
         self.H, self.E, self.k, self.el = H, E, k, E // self.world
+        self.T_max = T_max
         self.device = device or (router_w.device if router_w is not None else None)
         if backend is None and (router_w is None or local_w13 is None or local_w2 is None):
             raise ValueError("router_w, local_w13 and local_w2 are required for the library backend")
@@ -187,36 +203,53 @@ class ExpertParallelFfn:
     def _key(self, step: int, rank: int) -> str:
         return f"afd_ep/{step}/{rank}"
 
+    def _state_key(self, step: int) -> str:
+        return f"afd_ep/{step}/state"
+
+    def _missing(self, step: int) -> list:
+        missing = []
+        for r in range(self.world):
+            try:
+                if not self.liveness.check([self._key(step, r)]):
+                    missing.append(r)
+            except Exception:
+                missing.append(r)
+        return missing
+
     def check_peers(self) -> None:
         """Host-side check that every rank reached this step (no-op without a liveness store)."""
         st = self.liveness
         if st is None:
             return
         step = self.step
-        st.set(self._key(step, self.rank), "1")
         keys = [self._key(step, r) for r in range(self.world)]
         try:
-            st.wait(keys, datetime.timedelta(seconds=self.liveness_timeout_s))
-        except Exception as e:
-            missing = []
-            for r in range(self.world):
-                try:
-                    if not st.check([self._key(step, r)]):
-                        missing.append(r)
-                except Exception:
-                    missing.append(r)
-            raise PeerLost(step, missing or list(range(self.world))) from e
-        if step >= 2:
-            # every rank has set its key for step - 1, so all are done waiting on step - 2
+            st.set(self._key(step, self.rank), "1")
             try:
-                st.delete_key(self._key(step - 2, self.rank))
+                st.wait(keys, datetime.timedelta(seconds=self.liveness_timeout_s))
+                arrived = True
             except Exception:
-                pass
+                arrived = False
+            # one decision per step, taken by whichever rank gets there first
+            state = st.compare_set(self._state_key(step), "", "go" if arrived else "abort")
+        except Exception as e:                   # the store itself is gone
+            raise PeerLost(step, list(range(self.world))) from e
+        if bytes(state) != b"go":
+            raise PeerLost(step, self._missing(step))
+        if step >= 2:
+            # every rank has decided step - 1, so none still reads the keys of step - 2
+            for k in (self._key(step - 2, self.rank), self._state_key(step - 2)):
+                try:
+                    st.delete_key(k)
+                except Exception:
+                    pass
         self.step = step + 1
 
     def forward(self, hidden: torch.Tensor) -> torch.Tensor:
-        self.check_peers()
         T, H, k = hidden.shape[0], self.H, self.k
+        if T > self.T_max:
+            raise ValueError(f"micro-batch of {T} tokens exceeds T_max = {self.T_max}")
+        self.check_peers()
         b, g = self.backend, self.group
         idx, w = b.route(hidden, T)
         counts, pos, rows = b.dispatch(hidden, idx, T)

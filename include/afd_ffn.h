@@ -84,7 +84,8 @@ typedef struct {             /* all DEVICE pointers, 16-byte aligned, borrowed, 
 
 typedef struct afd_ffn_handle afd_ffn_handle;
 
-/* Create a handle on the current device: validates cfg and weights (host-side checks come
+/* Create a handle for one MoE layer of the FFN service (vLLM AFD Plugin page, section 系統架構,
+ * "2. FFN Service") on the current device: validates cfg and weights (host-side checks come
  * first and touch no device), allocates the workspace for T_max tokens and encodes the TMA
  * descriptors of the weights.  The handle also derives, once, what its kernels read instead of
  * the caller's tensors: the router weights as three bf16 planes (hi + mid + lo = Wr to ~2^-27),
@@ -97,12 +98,16 @@ int afd_ffn_create(const afd_ffn_cfg *cfg, const afd_ffn_weights *weights, afd_f
 /* Free the workspace and the handle (after synchronising the device).  NULL is a no-op. */
 void afd_ffn_destroy(afd_ffn_handle *h);
 
-/* Router, top-k and gate weights.  hidden [T][H] bf16 -> topk_idx [T][k] int32 (descending
- * logit order) and topk_w [T][k] fp32 (softmax over the selected logits).  0 <= T <= T_max. */
+/* Router, top-k and gate weights: the routing computation the FFN side runs for each token
+ * (vLLM AFD Plugin page, section Attention-FFN 解耦的原理), picking a few of the layer's many
+ * experts per token (LLM 推理提速: Attention与FFN分离AFD方, section 一个在啃带宽，一个在吃算力).
+ * hidden [T][H] bf16 -> topk_idx [T][k] int32 (descending logit order) and topk_w [T][k] fp32
+ * (softmax over the selected logits).  0 <= T <= T_max. */
 int afd_ffn_route(afd_ffn_handle *h, const void *hidden, int32_t T,
                   int32_t *topk_idx, float *topk_w, void *stream);
 
-/* Dispatch order and dispatched rows.  From topk_idx [T][k]:
+/* Dispatch order and dispatched rows: each token's hidden state is sent to the experts it
+ * chose (A/F 分离 page, section 机制, the dispatch step).  From topk_idx [T][k]:
  *   counts [E]      rows per expert
  *   offsets[E+1]    exclusive prefix sum of counts (offsets[E] = number of valid pairs)
  *   pos    [T][k]   dispatched row of pair (t,j): expert-major, ascending t inside an expert;
@@ -113,20 +118,24 @@ int afd_ffn_route(afd_ffn_handle *h, const void *hidden, int32_t T,
 int afd_ffn_permute(afd_ffn_handle *h, const void *hidden, const int32_t *topk_idx, int32_t T,
                     int32_t *counts, int32_t *offsets, int32_t *pos, int32_t *src, void *stream);
 
-/* Expert FFNs on the rows dispatched by the last afd_ffn_permute of this handle, grouped by
+/* Expert FFNs -- each expert is a large matrix product (A/F 分离 page, section 为什么要拆) --
+ * on the rows dispatched by the last afd_ffn_permute of this handle, grouped by
  * `offsets` [E+1] (device).  Writes the handle's internal output rows (fp32; bf16 on the W8A8
  * path); when non-NULL also copies them out as fp32: Y [T*k][H] (row p = the output of
  * dispatched row p, unweighted) and Ys [T][H] (shared expert; must be NULL when n_shared == 0). */
 int afd_ffn_expert_gemm(afd_ffn_handle *h, const int32_t *offsets, int32_t T,
                         float *Y, float *Ys, void *stream);
 
-/* Weighted combine of the handle's internal expert outputs:
+/* Weighted combine of the handle's internal expert outputs, back in token order (A/F 分离
+ * page, section 机制, the combine step):
  * out[t] = sum_j topk_w[t][j] * Y[pos[t][j]] + Ys[t], fp32 sum in j order, bf16 out [T][H]. */
 int afd_ffn_combine(afd_ffn_handle *h, const float *topk_w, const int32_t *pos, int32_t T,
                     void *out, void *stream);
 
-/* The whole layer: hidden [T][H] bf16 -> out [T][H] bf16 (route, permute, expert GEMMs,
- * combine).  No host synchronisation, no allocation: capturable in a CUDA graph. */
+/* The whole layer, the FFN service's compute_ffn_output() for one micro-batch (vLLM AFD
+ * Plugin page, section 系統架構, "2. FFN Service"): hidden [T][H] bf16 -> out [T][H] bf16
+ * (route, permute, expert GEMMs, combine).  No host synchronisation, no allocation:
+ * capturable in a CUDA graph. */
 int afd_ffn_forward(afd_ffn_handle *h, const void *hidden, int32_t T, void *out, void *stream);
 
 /* The whole layer on HOST buffers: copies hidden_host [T][H] bf16 to the device, runs
@@ -191,6 +200,9 @@ const char *afd_ffn_strerror(int status);
  * Every call on a device shares the one array: calls that can overlap on the GPU (different
  * streams without ordering between them) race on it and must be serialised by the caller.
  * Nothing in the array needs clearing: each call overwrites every element it reads.
+ * The looked-up address is kept for the life of the process: it does not survive a
+ * cudaDeviceReset (or any other teardown of the device's primary context), after which this
+ * call must not be used on that device.
  * CUDA failures return AFD_ERR_CUDA; the cudaError_t is afd_ffn_last_cuda_error(NULL). */
 #define AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS (1 << 20)
 int afd_ffn_route_static(const void *hidden, const float *router_w, const float *router_bias,

@@ -18,13 +18,15 @@ class Layer:
     """Seeded inputs of ``cfg`` on host and device plus a library handle (T_max = cfg.T)."""
 
     def __init__(self, cfg: synth.MoEConfig, T_max: int | None = None, hidden=None, bias=None,
-                 redraws=None):
+                 redraws=None, edit_experts=None):
         self.cfg = cfg
         self.fp8 = cfg.dtype == "fp8"
         self.hidden = synth.gen_hidden(cfg, redraws=redraws) if hidden is None else hidden
         self.Wr, b = synth.gen_router(cfg)
         self.bias = b if bias is None else bias
         self.experts = synth.gen_experts(cfg)
+        if edit_experts is not None:            # a test's change to the weights, before upload
+            edit_experts(self.experts)
         dev = {k: v.cuda() for k, v in self.experts.items()}
         dev["router_w"] = self.Wr.cuda()
         if self.bias is not None:

@@ -1,0 +1,42 @@
+"""Host-side accounting of bench.py (CPU only): which peak bounds each workload's dominant
+kernel, its algorithmic bytes and FLOPs, and the library launches per forward."""
+import numpy as np
+
+import bench
+import synth
+
+
+def _acct(name):
+    cfg = synth.CONFIGS[name]
+    counts = np.full(cfg.E, cfg.T * cfg.k // cfg.E)       # every routed expert touched
+    return cfg, bench.algorithmic(cfg, counts)
+
+
+def test_decode_shape_is_hbm_bound_on_the_expert_weights():
+    cfg, acct = _acct("dsv3_256")
+    assert acct["touched_experts"] == 257
+    assert acct["weight_bytes"] == 257 * 3 * 7168 * 2048 * 2
+    roof, path = bench.rooflines(cfg, acct, ms=3.5, kernel_ms=3.45)
+    assert roof["bound"] == "hbm" and roof["unit"] == "GB/s"
+    assert roof["algorithmic_bytes_per_launch"] == acct["weight_bytes"]   # weights only
+    assert abs(roof["achieved"] - acct["weight_bytes"] / 3.45e-3 / 1e9) < 0.1
+    assert path["t_hbm_ms"] > path["t_tensor_ms"]
+    assert bench.launches_per_step(cfg) == 8
+
+
+def test_w8a8_large_chunk_gate_up_is_tensor_bound():
+    cfg, acct = _acct("w8a8_8192")
+    roof, path = bench.rooflines(cfg, acct, ms=4.5, kernel_ms=2.3)
+    rows = cfg.T * cfg.k + cfg.T
+    assert roof["algorithmic_flops_per_launch"] == 4 * cfg.H * cfg.I * rows
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert roof["peak"] == 2 * bench.load_peaks()[0]["bf16_tflops"]         # e4m3 = 2 x bf16
+    assert bench.launches_per_step(cfg) == 11                             # T >= 2048: +1
+
+
+def test_bf16_large_micro_batch_gate_up_is_hbm_bound():
+    cfg, acct = _acct("dsv3_4096")
+    roof, _ = bench.rooflines(cfg, acct, ms=5.0, kernel_ms=2.7)
+    assert roof["bound"] == "hbm"
+    assert roof["algorithmic_bytes_per_launch"] == 257 * 2 * 2048 * 7168 * 2
+    assert bench.launches_per_step(cfg) == 10

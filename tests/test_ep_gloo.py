@@ -236,3 +236,70 @@ def test_liveness_checked_steps_match_the_oracle():
         assert p.exitcode == 0
     for rank, worst, steps in sorted(q.get(timeout=10) for _ in range(2)):
         assert worst <= 1e-12 and steps == 4, (rank, worst, steps)
+
+
+def _slow_worker(rank, world, port, q):
+    """Both ranks take one step; then rank 1 sleeps past rank 0's liveness timeout (alive, only
+    slow).  The step must be aborted consistently: rank 0 gives up and reports rank 1 missing,
+    rank 1 arrives late, finds the step decided as aborted and raises too -- neither enters the
+    exchange, so no rank is left waiting inside a collective."""
+    import datetime
+    import time
+    from ep_support import OracleRowsBackend
+    from ffn_side_expert_b200.ep import PeerLost
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    try:
+        store = dist.TCPStore("127.0.0.1", port + 1, world, is_master=(rank == 0),
+                              timeout=datetime.timedelta(seconds=20))
+        Wr, experts = _weights()
+        el = E // world
+        backend = _CountingBackend(OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K,
+                                                     local_experts=experts[rank * el:(rank + 1) * el],
+                                                     shared=experts[E]))
+        ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend, liveness=store,
+                               liveness_timeout_s=1.5)
+        hidden = torch.from_numpy(np.random.default_rng(3 + rank).normal(0, 1, (6, H)))
+        ep.forward(hidden)
+        if rank == 1:
+            time.sleep(4.0)
+        try:
+            ep.forward(hidden)
+            outcome = "no error"
+        except PeerLost as e:
+            outcome = f"PeerLost {e.missing}"
+        q.put((rank, outcome, backend.routed))
+        dist.barrier()                                 # both ranks are still alive and in step
+    finally:
+        dist.destroy_process_group()
+
+
+def test_a_slow_rank_aborts_the_step_on_every_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 22600 + 2 * (os.getpid() % 500)
+    procs = [ctx.Process(target=_slow_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(90)
+        assert p.exitcode == 0
+    res = dict((r, (o, n)) for r, o, n in (q.get(timeout=10) for _ in range(2)))
+    assert res[0] == ("PeerLost [1]", 1)               # gave up waiting for rank 1
+    assert res[1] == ("PeerLost []", 1)                # arrived late: the step was already aborted
+
+
+def test_a_micro_batch_above_T_max_is_refused_before_any_work():
+    class _Group:
+        pass
+
+    class _Never:
+        def route(self, *a):
+            raise AssertionError("routed a micro-batch above T_max")
+
+    import ffn_side_expert_b200.ep as epmod
+    ep = ExpertParallelFfn.__new__(ExpertParallelFfn)
+    ep.world, ep.rank, ep.H, ep.E, ep.k, ep.el, ep.T_max = 1, 0, H, E, K, E, 16
+    ep.backend, ep.group, ep.liveness, ep.step = _Never(), None, None, 0
+    with pytest.raises(ValueError, match="T_max"):
+        epmod.ExpertParallelFfn.forward(ep, torch.zeros((17, H), dtype=torch.float64))

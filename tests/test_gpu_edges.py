@@ -198,3 +198,55 @@ def test_w8a8_wide_tiles():
         _check_layer(L, cfg.T, tol=FP8_TOL)
     finally:
         L.close()
+
+
+@pytest.mark.parametrize("shape", ["decode", "wide"])
+def test_large_gate_preactivations(shape):
+    # hidden rows scaled by 64 or 128 (exact in bf16; the logits scale exactly, so the margin redraws
+    # still hold): gate pre-activations z reach |z| > 90, where e^-z overflows fp32 and silu
+    # must still give z (z > 0) or -0 (z < 0), and the SwiGLU output reaches ~10^4-10^5 -- past
+    # the f16 range on the wide path, which stores each row with its power-of-two scale.
+    # decode: tiny (T*k <= 32 E, fused kernel, two-term bf16 act); wide: T*k > 32 E (f16 act)
+    base = (synth.CONFIGS["tiny"] if shape == "decode"
+            else synth.MoEConfig("wide", T=600, H=256, E=2, k=1, I=256, S=1, seed=24))
+    red = synth.load_redraws("tiny") if shape == "decode" else _redraws(base)
+    hidden = synth.gen_hidden(base, redraws=red) * (64 if shape == "decode" else 128)
+    L = Layer(base, hidden=hidden)
+    try:
+        x = moe._f64(hidden)
+        zmin, zmax, amax = 0.0, 0.0, 0.0
+        for e in range(base.E + base.S):
+            w13, _ = moe.expert_weights_f64(L.expert_fn(e))
+            z = x @ w13[:base.I].T
+            act = moe.silu(z) * (x @ w13[base.I:].T)
+            zmin, zmax, amax = min(zmin, z.min()), max(zmax, z.max()), max(amax, np.abs(act).max())
+        assert zmin < -90 and zmax > 90
+        if shape == "wide":
+            assert amax > 65504                              # past the f16 range
+        _check_layer(L, base.T)
+    finally:
+        L.close()
+
+
+def test_w8a8_zero_rows():
+    # W8A8 rows whose amax is 0 take the scale 1 on the GPU too: token 5 is an all-zero hidden
+    # row (its logits all tie at 0: experts 0 and 1, lower index first, weights 1/2), and expert 3
+    # has all-zero up rows, so every SwiGLU row it produces is zero
+    cfg = synth.MoEConfig("fp8s", T=64, H=512, E=8, k=2, I=256, S=1, dtype="fp8", seed=25)
+    hidden = synth.gen_hidden(cfg, redraws=_redraws(cfg))
+    hidden[5] = 0
+
+    def zero_up(ex):
+        ex["w13"][3, cfg.I:] = torch.zeros((cfg.I, cfg.H), dtype=torch.float32).to(torch.float8_e4m3fn)
+
+    L = Layer(cfg, hidden=hidden, edit_experts=zero_up)
+    try:
+        out = _check_layer(L, cfg.T, tol=FP8_TOL)
+        idx, w = L.route()
+        assert idx[5].tolist() == [0, 1] and w[5].tolist() == [0.5, 0.5]
+        assert (idx == 3).any()
+        ref = L.oracle()
+        assert np.all(ref["y_routed"][np.nonzero(ref["idx"] == 3)] == 0.0)
+        assert torch.isfinite(out.float()).all()
+    finally:
+        L.close()
