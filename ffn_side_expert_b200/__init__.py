@@ -79,6 +79,9 @@ _SIGNATURES = {
     "afd_ffn_expert_rows": (ctypes.c_int, [_P, _P, _P, _I, _P, _P]),
     "afd_ffn_copy_row_blocks": (ctypes.c_int, [_P, _P, _P, _I, _I, _P]),
     "afd_ffn_combine_rows": (ctypes.c_int, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "afd_ffn_dispatch_rows_fp8": (ctypes.c_int, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "afd_ffn_expert_rows_fp8": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _P]),
+    "afd_ffn_combine_rows_bf16": (ctypes.c_int, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "afd_ffn_rows_error": (ctypes.c_int, []),
     "afd_ffn_get_info": (ctypes.c_int, [_P, ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(ctypes.c_int32)]),
     "afd_ffn_check_bounded_wait": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int64)]),
@@ -241,6 +244,23 @@ def afd_ffn_expert_rows(h, rows, counts, n_rows, Y, stream=None) -> int:
 
 def afd_ffn_copy_row_blocks(src, dst, blocks, n_blocks, row_bytes, stream=None) -> int:
     return _lib.afd_ffn_copy_row_blocks(_ptr(src), _ptr(dst), _ptr(blocks), n_blocks, row_bytes, _stream(stream))
+
+
+def afd_ffn_dispatch_rows_fp8(hidden, topk_idx, T, k, E, H, with_shared, counts, offsets, pos, src, rows,
+                              row_scale, scratch, stream=None) -> int:
+    return _lib.afd_ffn_dispatch_rows_fp8(_ptr(hidden), _ptr(topk_idx), T, k, E, H, with_shared, _ptr(counts),
+                                          _ptr(offsets), _ptr(pos), _ptr(src), _ptr(rows), _ptr(row_scale),
+                                          _ptr(scratch), _stream(stream))
+
+
+def afd_ffn_expert_rows_fp8(h, rows, row_scale, counts, n_rows, Y, stream=None) -> int:
+    return _lib.afd_ffn_expert_rows_fp8(h, _ptr(rows), _ptr(row_scale), _ptr(counts), n_rows, _ptr(Y),
+                                        _stream(stream))
+
+
+def afd_ffn_combine_rows_bf16(Y, Ys, topk_w, pos, T, k, H, out, stream=None) -> int:
+    return _lib.afd_ffn_combine_rows_bf16(_ptr(Y), _ptr(Ys), _ptr(topk_w), _ptr(pos), T, k, H, _ptr(out),
+                                          _stream(stream))
 
 
 def afd_ffn_combine_rows(Y, Ys, topk_w, pos, T, k, H, out, stream=None) -> int:

@@ -1181,6 +1181,74 @@ extern "C" int afd_ffn_dispatch_rows(const void* hidden, const int32_t* topk_idx
   return AFD_OK;
 }
 
+extern "C" int afd_ffn_dispatch_rows_fp8(const void* hidden, const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
+                                         int32_t H, int32_t with_shared, int32_t* counts, int32_t* offsets,
+                                         int32_t* pos, int32_t* src, void* rows, float* row_scale, int32_t* scratch,
+                                         void* stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1 || E > kMaxExperts || k > E || H < 16 || H % 16 != 0) return AFD_ERR_INVALID_ARG;
+  if (with_shared != 0 && with_shared != 1) return AFD_ERR_INVALID_ARG;
+  if (!counts || !offsets || !scratch) return AFD_ERR_INVALID_ARG;
+  if (T > 0 && (!hidden || !topk_idx || !pos || !src || !rows || !row_scale || !aligned16(hidden) || !aligned16(rows)))
+    return AFD_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * (k + 1) > (1LL << 30)) return AFD_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  int st = rows_err_word(&err);
+  if (st != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nchunks = (T + kChunkTokens - 1) / kChunkTokens;
+  int32_t* chunk_counts = scratch;
+  int32_t* chunk_base = scratch + static_cast<size_t>(nchunks) * E;
+  if (T > 0)
+    dispatch_count_kernel<<<nchunks, kCountThreads, 0, s>>>(topk_idx, T, k, E, pos, chunk_counts, err);
+  dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(chunk_counts, nchunks, E, counts, offsets, chunk_base);
+  if (T > 0)
+    gather_rows_kernel<true><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), topk_idx, chunk_base, pos,
+                                               src, T, k, E, H, with_shared, static_cast<uint8_t*>(rows), row_scale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_expert_rows_fp8(afd_ffn_handle* h, const void* rows, const float* row_scale,
+                                       const int32_t* counts, int32_t n_rows, void* Y, void* stream) {
+  if (!h) return AFD_ERR_INVALID_ARG;
+  const afd_ffn_cfg& c = h->cfg;
+  if (c.k != 1 || c.n_shared != 0 || !h->fp8) return AFD_ERR_UNSUPPORTED;
+  int st = check_T(h, n_rows);
+  if (st != AFD_OK) return st;
+  if (n_rows == 0) return AFD_OK;
+  if (!rows || !row_scale || !counts || !Y || !aligned16(rows) || !aligned16(Y)) return AFD_ERR_INVALID_ARG;
+  if ((st = check_device(h)) != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  const size_t H = c.H;
+  AFD_CUDA(h, cudaMemcpyAsync(h->xp, rows, static_cast<size_t>(n_rows) * H, cudaMemcpyDeviceToDevice, s));
+  AFD_CUDA(h, cudaMemcpyAsync(h->xscale, row_scale, static_cast<size_t>(n_rows) * 4, cudaMemcpyDeviceToDevice, s));
+  dispatch_scan_kernel<<<1, kMaxExperts, 0, s>>>(counts, 1, c.E, h->counts, h->offsets, h->chunk_base);
+  AFD_CUDA(h, cudaGetLastError());
+  if ((st = run_expert_gemm(h, h->offsets, n_rows, s)) != AFD_OK) return st;
+  AFD_CUDA(h, cudaMemcpyAsync(Y, h->Y, static_cast<size_t>(n_rows) * H * 2, cudaMemcpyDeviceToDevice, s));
+  return AFD_OK;
+}
+
+extern "C" int afd_ffn_combine_rows_bf16(const void* Y, const void* Ys, const float* topk_w, const int32_t* pos,
+                                         int32_t T, int32_t k, int32_t H, void* out, void* stream) {
+  if (T < 0 || k < 1 || k > 32 || H < 4 || H % 4 != 0) return AFD_ERR_INVALID_ARG;
+  if (T == 0) return AFD_OK;
+  if (!Y || !topk_w || !pos || !out || !aligned16(Y) || !aligned16(out) || (Ys && !aligned16(Ys)))
+    return AFD_ERR_INVALID_ARG;
+  int* err = nullptr;
+  int st = rows_err_word(&err);
+  if (st != AFD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  combine_kernel<__nv_bfloat16><<<T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(Y),
+                                                  static_cast<const __nv_bfloat16*>(Ys), topk_w, pos, T, k, H, T * k,
+                                                  Ys ? 1 : 0, static_cast<__nv_bfloat16*>(out), err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(nullptr, e);
+  return AFD_OK;
+}
+
 extern "C" int afd_ffn_expert_rows(afd_ffn_handle* h, const void* rows, const int32_t* counts, int32_t n_rows,
                                    float* Y, void* stream) {
   if (!h) return AFD_ERR_INVALID_ARG;
@@ -1208,12 +1276,19 @@ extern "C" int afd_ffn_expert_rows(afd_ffn_handle* h, const void* rows, const in
 
 extern "C" int afd_ffn_copy_row_blocks(const void* src, void* dst, const int32_t* blocks, int32_t n_blocks,
                                        int32_t row_bytes, void* stream) {
-  if (n_blocks < 0 || row_bytes < 16 || row_bytes % 16 != 0) return AFD_ERR_INVALID_ARG;
+  if (n_blocks < 0 || row_bytes < 4 || row_bytes % 4 != 0) return AFD_ERR_INVALID_ARG;
   if (n_blocks == 0) return AFD_OK;
-  if (!src || !dst || !blocks || !aligned16(src) || !aligned16(dst)) return AFD_ERR_INVALID_ARG;
+  const bool wide = row_bytes % 16 == 0;
+  const uintptr_t mis = (reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & (wide ? 15u : 3u);
+  if (!src || !dst || !blocks || mis) return AFD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  copy_row_blocks_kernel<<<dim3(static_cast<unsigned>(n_blocks), 16), 256, 0, s>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), blocks, row_bytes / 16);
+  const dim3 grid(static_cast<unsigned>(n_blocks), 16);
+  if (wide)
+    copy_row_blocks_kernel<uint4><<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), blocks,
+                                                        row_bytes / 16);
+  else
+    copy_row_blocks_kernel<uint32_t><<<grid, 256, 0, s>>>(static_cast<const uint32_t*>(src),
+                                                           static_cast<uint32_t*>(dst), blocks, row_bytes / 4);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;

@@ -89,16 +89,18 @@ combine_kernel(const YT* __restrict__ Y, const YT* __restrict__ Ys, const float*
 }
 
 // Copy blocks of rows: block b moves blocks[3b+2] rows of row_bytes from row blocks[3b] of src
-// to row blocks[3b+1] of dst.  blockIdx.x = block, blockIdx.y splits its rows; 16-byte moves.
+// to row blocks[3b+1] of dst.  blockIdx.x = block, blockIdx.y splits its rows; moves of V
+// (16 bytes, or 4 for rows that are not a multiple of 16 bytes, such as per-row scales).
+template <typename V>
 __global__ void __launch_bounds__(256)
-copy_row_blocks_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ blocks,
+copy_row_blocks_kernel(const V* __restrict__ src, V* __restrict__ dst, const int32_t* __restrict__ blocks,
                        int row_vecs) {
   const int b = blockIdx.x;
   const size_t s0 = static_cast<size_t>(blocks[3 * b]), d0 = static_cast<size_t>(blocks[3 * b + 1]);
   const int rows = blocks[3 * b + 2];
   for (int r = blockIdx.y; r < rows; r += gridDim.y) {
-    const uint4* sr = src + (s0 + r) * row_vecs;
-    uint4* dr = dst + (d0 + r) * row_vecs;
+    const V* sr = src + (s0 + r) * row_vecs;
+    V* dr = dst + (d0 + r) * row_vecs;
     for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) dr[v] = sr[v];
   }
 }

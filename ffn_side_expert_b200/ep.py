@@ -11,8 +11,13 @@ hold its experts, and their outputs come back for the weighted combine; the page
   2. exchange the per-expert row counts, then the rows (all-to-all-v);
   3. regroup the received rows from [source rank][local expert] to [local expert][source rank]
      and run the local experts;
-  4. restore the received order and send the fp32 outputs back (all-to-all-v);
+  4. restore the received order and send the outputs back (all-to-all-v);
   5. combine: out[t] = sum_j w[t,j] * Y[pos[t,j]] + shared(hidden[t]).
+
+Precision on the wire: bf16 weights send bf16 rows and get fp32 outputs back.  W8A8 weights
+send each dispatched row as its e4m3 codes plus one fp32 scale -- the quantised hidden row
+the experts consume anyway, so the exchange adds no error and its dispatch bytes are the
+page's FP8 account plus 4 bytes of scale per row -- and get bf16 outputs back.
 
 Every arithmetic step runs in the library's kernels (ExpertParallelFfn's default backend);
 torch.distributed moves the bytes (NCCL between GPUs).  The backend is a parameter only so that
@@ -27,7 +32,8 @@ import torch
 import torch.distributed as dist
 
 from . import (AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS, AFD_OK, AfdError, AfdFfn, afd_ffn_combine_rows,
-               afd_ffn_copy_row_blocks, afd_ffn_dispatch_rows, afd_ffn_expert_rows, afd_ffn_route_static)
+               afd_ffn_combine_rows_bf16, afd_ffn_copy_row_blocks, afd_ffn_dispatch_rows, afd_ffn_dispatch_rows_fp8,
+               afd_ffn_expert_rows, afd_ffn_expert_rows_fp8, afd_ffn_route_static)
 
 
 def block_tables(recv_counts: torch.Tensor):
@@ -67,10 +73,24 @@ def block_tables(recv_counts: torch.Tensor):
 class WireBytes:
     """Bytes one forward moved through the exchange on this rank."""
     dispatch_sent: int      # rows sent for dispatch (to every rank, this one included) x row bytes
+                            # (W8A8: e4m3 codes + the fp32 row scale)
     dispatch_remote: int    # ... of which to other ranks
-    combine_sent: int       # expert outputs sent back (fp32 rows)
+    combine_sent: int       # expert outputs sent back (fp32 rows; bf16 on the W8A8 path)
     combine_remote: int
     tokens: int
+    dispatch_rows: int = 0  # rows sent for dispatch (T*k when every pair is valid)
+
+
+@dataclass
+class Dispatched:
+    """One rank's dispatch: per-expert counts, each pair's row, the rows to send (expert-major)
+    and their per-row scales (W8A8; None otherwise); `shared` is backend data for the shared
+    expert (the CUDA W8A8 backend keeps the token-order quantised rows there)."""
+    counts: torch.Tensor
+    pos: torch.Tensor
+    rows: torch.Tensor
+    scales: torch.Tensor | None = None
+    shared: object = None
 
 
 class PeerLost(RuntimeError):
@@ -83,20 +103,29 @@ class PeerLost(RuntimeError):
 
 
 class CudaRowsBackend:
-    """The library's kernels for every step of the expert-parallel forward on one rank."""
+    """The library's kernels for every step of the expert-parallel forward on one rank.
+
+    fp8: the expert weights are e4m3 (local_w13_scale / local_w2_scale and the shared scales
+    hold their per-output-channel fp32 scales); rows travel as e4m3 codes + fp32 row scales and
+    outputs as bf16."""
 
     def __init__(self, *, H, E, k, I, T_max, world, router_w, router_bias, local_w13, local_w2,
-                 shared_w13, shared_w2, device):
-        self.H, self.E, self.k, self.device = H, E, k, device
+                 shared_w13, shared_w2, device, fp8=False, local_w13_scale=None, local_w2_scale=None,
+                 shared_w13_scale=None, shared_w2_scale=None):
+        self.H, self.E, self.k, self.device, self.fp8 = H, E, k, device, fp8
         self.router_w, self.router_bias = router_w, router_bias
         el = E // world
         dummy_router = torch.zeros((el, H), dtype=torch.float32, device=device)  # unused by expert_rows
-        self.local = AfdFfn(T_max=world * T_max * k, H=H, E=el, k=1, I=I, n_shared=0, fp8=False,
-                            weights={"router_w": dummy_router, "w13": local_w13, "w2": local_w2})
+        wl = {"router_w": dummy_router, "w13": local_w13, "w2": local_w2}
+        if fp8:
+            wl.update(w13_scale=local_w13_scale, w2_scale=local_w2_scale)
+        self.local = AfdFfn(T_max=world * T_max * k, H=H, E=el, k=1, I=I, n_shared=0, fp8=fp8, weights=wl)
         self.shared = None
         if shared_w13 is not None:
-            self.shared = AfdFfn(T_max=T_max, H=H, E=1, k=1, I=I, n_shared=0, fp8=False,
-                                 weights={"router_w": dummy_router[:1], "w13": shared_w13[None], "w2": shared_w2[None]})
+            ws = {"router_w": dummy_router[:1], "w13": shared_w13[None], "w2": shared_w2[None]}
+            if fp8:
+                ws.update(w13_scale=shared_w13_scale[None], w2_scale=shared_w2_scale[None])
+            self.shared = AfdFfn(T_max=T_max, H=H, E=1, k=1, I=I, n_shared=0, fp8=fp8, weights=ws)
         self.scratch = torch.empty(2 * ((T_max + 127) // 128) * E, dtype=torch.int32, device=device)
         self.route_chunk = max(1, AFD_FFN_ROUTE_STATIC_SCRATCH_FLOATS // E)
         self.keep = [dummy_router]
@@ -117,39 +146,61 @@ class CudaRowsBackend:
                                           self.k, idx[t0:t0 + n], w[t0:t0 + n]), "afd_ffn_route_static")
         return idx, w
 
-    def dispatch(self, hidden, idx, T):
+    def dispatch(self, hidden, idx, T) -> Dispatched:
         counts = torch.empty(self.E, dtype=torch.int32, device=self.device)
         offsets = torch.empty(self.E + 1, dtype=torch.int32, device=self.device)
         pos = torch.empty((T, self.k), dtype=torch.int32, device=self.device)
         src = torch.empty(max(T * self.k, 1), dtype=torch.int32, device=self.device)
-        rows = torch.empty((max(T * self.k, 1), self.H), dtype=torch.bfloat16, device=self.device)
-        self._ok(afd_ffn_dispatch_rows(hidden, idx, T, self.k, self.E, self.H, counts, offsets, pos, src, rows,
-                                       self.scratch), "afd_ffn_dispatch_rows")
-        return counts, pos, rows
+        if not self.fp8:
+            rows = torch.empty((max(T * self.k, 1), self.H), dtype=torch.bfloat16, device=self.device)
+            self._ok(afd_ffn_dispatch_rows(hidden, idx, T, self.k, self.E, self.H, counts, offsets, pos, src, rows,
+                                           self.scratch), "afd_ffn_dispatch_rows")
+            return Dispatched(counts, pos, rows)
+        # the T token-order rows of the shared expert follow the dispatched ones
+        ws = 1 if self.shared is not None else 0
+        n = max(T * (self.k + ws), 1)
+        rows = torch.empty((n, self.H), dtype=torch.uint8, device=self.device)
+        scales = torch.empty(n, dtype=torch.float32, device=self.device)
+        self._ok(afd_ffn_dispatch_rows_fp8(hidden, idx, T, self.k, self.E, self.H, ws, counts, offsets, pos, src,
+                                           rows, scales, self.scratch), "afd_ffn_dispatch_rows_fp8")
+        tk = T * self.k
+        return Dispatched(counts, pos, rows[:max(tk, 1)], scales[:max(tk, 1)],
+                          shared=(rows[tk:], scales[tk:]) if ws else None)
 
     def copy_blocks(self, src, dst, blocks, row_bytes):
         if blocks.shape[0]:
             b = blocks.to(self.device)
             self._ok(afd_ffn_copy_row_blocks(src, dst, b, b.shape[0], row_bytes), "afd_ffn_copy_row_blocks")
 
-    def experts(self, rows, per_expert, n):
-        Y = torch.empty((max(n, 1), self.H), dtype=torch.float32, device=self.device)
+    def experts(self, rows, scales, per_expert, n):
+        Y = torch.empty((max(n, 1), self.H), dtype=torch.bfloat16 if self.fp8 else torch.float32,
+                        device=self.device)
         if n:
             cnt = per_expert.to(self.device)
-            self._ok(afd_ffn_expert_rows(self.local.h, rows, cnt, n, Y), "afd_ffn_expert_rows")
+            if self.fp8:
+                self._ok(afd_ffn_expert_rows_fp8(self.local.h, rows, scales, cnt, n, Y), "afd_ffn_expert_rows_fp8")
+            else:
+                self._ok(afd_ffn_expert_rows(self.local.h, rows, cnt, n, Y), "afd_ffn_expert_rows")
         return Y
 
-    def shared_expert(self, hidden, T):
+    def shared_expert(self, hidden, T, d: Dispatched):
         if self.shared is None:
             return None
-        Ys = torch.empty((max(T, 1), self.H), dtype=torch.float32, device=self.device)
         cnt = torch.tensor([T], dtype=torch.int32, device=self.device)
+        if self.fp8:
+            Ys = torch.empty((max(T, 1), self.H), dtype=torch.bfloat16, device=self.device)
+            if T:
+                self._ok(afd_ffn_expert_rows_fp8(self.shared.h, d.shared[0], d.shared[1], cnt, T, Ys),
+                         "afd_ffn_expert_rows_fp8 (shared)")
+            return Ys
+        Ys = torch.empty((max(T, 1), self.H), dtype=torch.float32, device=self.device)
         self._ok(afd_ffn_expert_rows(self.shared.h, hidden, cnt, T, Ys), "afd_ffn_expert_rows (shared)")
         return Ys
 
     def combine(self, Y, Ys, w, pos, T):
         out = torch.empty((max(T, 1), self.H), dtype=torch.bfloat16, device=self.device)
-        self._ok(afd_ffn_combine_rows(Y, Ys, w, pos, T, self.k, self.H, out), "afd_ffn_combine_rows")
+        fn = afd_ffn_combine_rows_bf16 if self.fp8 else afd_ffn_combine_rows
+        self._ok(fn(Y, Ys, w, pos, T, self.k, self.H, out), fn.__name__)
         return out[:T]
 
     def close(self):
@@ -182,7 +233,8 @@ class ExpertParallelFfn:
 
     def __init__(self, *, H, E, k, I, T_max, router_w=None, router_bias=None, local_w13=None, local_w2=None,
                  shared_w13=None, shared_w2=None, group=None, backend=None, device=None,
-                 liveness=None, liveness_timeout_s: float = 5.0):
+                 liveness=None, liveness_timeout_s: float = 5.0, local_w13_scale=None, local_w2_scale=None,
+                 shared_w13_scale=None, shared_w2_scale=None):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -193,9 +245,12 @@ class ExpertParallelFfn:
         self.device = device or (router_w.device if router_w is not None else None)
         if backend is None and (router_w is None or local_w13 is None or local_w2 is None):
             raise ValueError("router_w, local_w13 and local_w2 are required for the library backend")
+        fp8 = local_w13 is not None and local_w13.dtype == torch.float8_e4m3fn
         self.backend = backend or CudaRowsBackend(
             H=H, E=E, k=k, I=I, T_max=T_max, world=self.world, router_w=router_w, router_bias=router_bias,
-            local_w13=local_w13, local_w2=local_w2, shared_w13=shared_w13, shared_w2=shared_w2, device=self.device)
+            local_w13=local_w13, local_w2=local_w2, shared_w13=shared_w13, shared_w2=shared_w2, device=self.device,
+            fp8=fp8, local_w13_scale=local_w13_scale, local_w2_scale=local_w2_scale,
+            shared_w13_scale=shared_w13_scale, shared_w2_scale=shared_w2_scale)
         self.last_wire: WireBytes | None = None
         self.liveness, self.liveness_timeout_s = liveness, liveness_timeout_s
         self.step = 0
@@ -252,9 +307,10 @@ class ExpertParallelFfn:
         self.check_peers()
         b, g = self.backend, self.group
         idx, w = b.route(hidden, T)
-        counts, pos, rows = b.dispatch(hidden, idx, T)
-        # 2. per-(rank, local expert) row counts, then the rows
-        send_c = counts.view(self.world, self.el).contiguous()
+        d = b.dispatch(hidden, idx, T)
+        rows, scales = d.rows, d.scales
+        # 2. per-(rank, local expert) row counts, then the rows (and their scales)
+        send_c = d.counts.view(self.world, self.el).contiguous()
         recv_c = torch.empty_like(send_c)
         dist.all_to_all_single(recv_c, send_c, group=g)
         send_c_h, recv_c_h = send_c.cpu(), recv_c.cpu()
@@ -263,26 +319,35 @@ class ExpertParallelFfn:
         n_send, n_recv = sum(send_split), sum(recv_split)
         recv_rows = torch.empty((max(n_recv, 1), H), dtype=rows.dtype, device=rows.device)
         dist.all_to_all_single(recv_rows[:n_recv], rows[:n_send], recv_split, send_split, group=g)
+        recv_scales = None
+        if scales is not None:
+            recv_scales = torch.empty(max(n_recv, 1), dtype=scales.dtype, device=scales.device)
+            dist.all_to_all_single(recv_scales[:n_recv], scales[:n_send], recv_split, send_split, group=g)
         # 3. local experts on the rows regrouped by expert
         to_grouped, to_received, per_expert = block_tables(recv_c_h)
         grouped = torch.empty_like(recv_rows)
         b.copy_blocks(recv_rows, grouped, to_grouped, H * rows.element_size())
-        Yg = b.experts(grouped, per_expert, n_recv)
+        grouped_scales = None
+        if recv_scales is not None:
+            grouped_scales = torch.empty_like(recv_scales)
+            b.copy_blocks(recv_scales, grouped_scales, to_grouped, scales.element_size())
+        Yg = b.experts(grouped, grouped_scales, per_expert, n_recv)
         # 4. outputs back in the order each source sent its rows
         Yr = torch.empty_like(Yg)
         b.copy_blocks(Yg, Yr, to_received, H * Yg.element_size())
         Yback = torch.empty((max(n_send, 1), H), dtype=Yg.dtype, device=Yg.device)
         dist.all_to_all_single(Yback[:n_send], Yr[:n_recv], send_split, recv_split, group=g)
         # 5. weighted combine with the shared expert
-        Ys = b.shared_expert(hidden, T)
-        out = b.combine(Yback, Ys, w, pos, T)
-        rb, yb = H * rows.element_size(), H * Yg.element_size()
+        Ys = b.shared_expert(hidden, T, d)
+        out = b.combine(Yback, Ys, w, d.pos, T)
+        rb = H * rows.element_size() + (scales.element_size() if scales is not None else 0)
+        yb = H * Yg.element_size()
         self.last_wire = WireBytes(
             dispatch_sent=n_send * rb,
             dispatch_remote=(n_send - send_split[self.rank]) * rb,
             combine_sent=n_recv * yb,
             combine_remote=(n_recv - recv_split[self.rank]) * yb,
-            tokens=T)
+            tokens=T, dispatch_rows=n_send)
         return out
 
     def close(self):

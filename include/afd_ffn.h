@@ -237,7 +237,8 @@ int afd_ffn_expert_rows(afd_ffn_handle *h, const void *rows, const int32_t *coun
 
 /* Move blocks of rows: block b copies blocks[3b+2] rows of row_bytes bytes from row blocks[3b]
  * of src to row blocks[3b+1] of dst (blocks: int32 [n_blocks][3], device).  Blocks must not
- * overlap in dst.  row_bytes a multiple of 16; src, dst 16-byte aligned. */
+ * overlap in dst.  row_bytes a multiple of 4 (per-row scales) with src, dst 4-byte aligned, or
+ * a multiple of 16 with src, dst 16-byte aligned (moved as 16-byte vectors). */
 int afd_ffn_copy_row_blocks(const void *src, void *dst, const int32_t *blocks, int32_t n_blocks,
                             int32_t row_bytes, void *stream);
 
@@ -247,6 +248,35 @@ int afd_ffn_copy_row_blocks(const void *src, void *dst, const int32_t *blocks, i
  * H multiple of 4; Y, Ys, out 16-byte aligned. */
 int afd_ffn_combine_rows(const float *Y, const float *Ys, const float *topk_w, const int32_t *pos,
                          int32_t T, int32_t k, int32_t H, void *out, void *stream);
+
+/* W8A8 form of the exchange, at the precision the A/F 分离 page counts its bytes in (section
+ * 深入推导 / 通信账: the dispatched hidden states travel as FP8).  The rows sent are exactly
+ * what the experts consume -- each token's hidden row quantised once to e4m3 with its fp32
+ * scale (row amax / 448, 1 for a zero row; round to nearest even, saturating) -- so sending
+ * them adds no error; the expert outputs come back as bf16 rows, the W8A8 layer's own output
+ * precision for the combine. */
+
+/* afd_ffn_dispatch_rows for the W8A8 path: the same counts, offsets, pos and src, and
+ * rows [T*k + with_shared*T][H] e4m3 + row_scale [T*k + with_shared*T] fp32: the quantised
+ * hidden rows in expert-major order, then (with_shared = 1) every token's row once, in token
+ * order, for a replicated shared expert.  hidden, rows 16-byte aligned; H a multiple of 16;
+ * scratch as for afd_ffn_dispatch_rows.  Asynchronous on `stream`. */
+int afd_ffn_dispatch_rows_fp8(const void *hidden, const int32_t *topk_idx, int32_t T, int32_t k, int32_t E,
+                              int32_t H, int32_t with_shared, int32_t *counts, int32_t *offsets, int32_t *pos,
+                              int32_t *src, void *rows, float *row_scale, int32_t *scratch, void *stream);
+
+/* afd_ffn_expert_rows for a W8A8 handle (k == 1, n_shared == 0): rows [n_rows][H] e4m3 with
+ * row_scale [n_rows] fp32, grouped by expert as counts [E] says -> Y [n_rows][H] bf16 (the W8A8
+ * expert outputs, SwiGLU rows quantised per row before the down projection as in
+ * afd_ffn_forward).  0 <= n_rows <= T_max; rows, Y 16-byte aligned.  Asynchronous. */
+int afd_ffn_expert_rows_fp8(afd_ffn_handle *h, const void *rows, const float *row_scale, const int32_t *counts,
+                            int32_t n_rows, void *Y, void *stream);
+
+/* afd_ffn_combine_rows on bf16 expert outputs: Y [T*k][H] bf16, Ys [T][H] bf16 or NULL; the same
+ * fp32 sum in j order with the shared row last, bf16 out [T][H].  H multiple of 4; Y, Ys, out
+ * 16-byte aligned. */
+int afd_ffn_combine_rows_bf16(const void *Y, const void *Ys, const float *topk_w, const int32_t *pos, int32_t T,
+                              int32_t k, int32_t H, void *out, void *stream);
 
 /* Synchronise the device; AFD_ERR_DEVICE_FLAG if an allocation-free call skipped invalid data
  * since the last check (the word is cleared), else AFD_OK. */

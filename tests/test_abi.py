@@ -81,13 +81,25 @@ def test_expert_parallel_calls_fail_fast_on_bad_arguments():
     assert afd.afd_ffn_dispatch_rows(A, A, 4, 2, 8, 256, A, A, A, A, A + 2, A) == afd.AFD_ERR_INVALID_ARG  # rows
     assert afd.afd_ffn_dispatch_rows(A, A, 4, 2, 8, 256, None, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG
     assert afd.afd_ffn_expert_rows(None, A, A, 4, A) == afd.AFD_ERR_INVALID_ARG
-    assert afd.afd_ffn_copy_row_blocks(A, A, A, 1, 8) == afd.AFD_ERR_INVALID_ARG                        # 8-byte rows
+    assert afd.afd_ffn_copy_row_blocks(A, A, A, 1, 6) == afd.AFD_ERR_INVALID_ARG                        # 6-byte rows
+    assert afd.afd_ffn_copy_row_blocks(A + 2, A, A, 1, 4) == afd.AFD_ERR_INVALID_ARG                    # 4-byte rows
+    assert afd.afd_ffn_copy_row_blocks(A + 4, A, A, 1, 32) == afd.AFD_ERR_INVALID_ARG                   # 16-byte moves
     assert afd.afd_ffn_copy_row_blocks(A, A, A, -1, 16) == afd.AFD_ERR_INVALID_ARG
     assert afd.afd_ffn_copy_row_blocks(A, A, A, 0, 16) == afd.AFD_OK                                    # nothing to do
     assert afd.afd_ffn_combine_rows(A, None, A, A, 4, 33, 256, A) == afd.AFD_ERR_INVALID_ARG            # k > 32
     assert afd.afd_ffn_combine_rows(A, None, A, A, 4, 2, 6, A) == afd.AFD_ERR_INVALID_ARG               # H % 4
     assert afd.afd_ffn_combine_rows(A, A + 4, A, A, 4, 2, 256, A) == afd.AFD_ERR_INVALID_ARG            # Ys align
     assert afd.afd_ffn_combine_rows(A, None, A, A, 0, 2, 256, A) == afd.AFD_OK                          # T = 0
+    # the W8A8 exchange
+    fp8d = afd.afd_ffn_dispatch_rows_fp8
+    assert fp8d(A, A, 4, 2, 8, 264, 1, A, A, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG       # H % 16
+    assert fp8d(A, A, 4, 2, 8, 256, 2, A, A, A, A, A, A, A) == afd.AFD_ERR_INVALID_ARG       # with_shared
+    assert fp8d(A, A, 4, 2, 8, 256, 1, A, A, A, A, A, None, A) == afd.AFD_ERR_INVALID_ARG    # no scales
+    assert fp8d(A, A, 4, 2, 8, 256, 1, A, A, A, A, A + 8, A, A) == afd.AFD_ERR_INVALID_ARG   # rows align
+    assert afd.afd_ffn_expert_rows_fp8(None, A, A, A, 4, A) == afd.AFD_ERR_INVALID_ARG
+    assert afd.afd_ffn_combine_rows_bf16(A, None, A, A, 4, 0, 256, A) == afd.AFD_ERR_INVALID_ARG      # k = 0
+    assert afd.afd_ffn_combine_rows_bf16(A, A + 2, A, A, 4, 2, 256, A) == afd.AFD_ERR_INVALID_ARG     # Ys align
+    assert afd.afd_ffn_combine_rows_bf16(A, None, A, A, 0, 2, 256, A) == afd.AFD_OK                   # T = 0
 
 
 def test_service_calls_fail_fast_without_a_handle():

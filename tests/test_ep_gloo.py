@@ -22,25 +22,32 @@ H, E, K, I = 16, 8, 2, 24
 TOKENS = {0: 12, 1: 9}
 
 
-def _weights():
+def _weights(fp8=False):
     rng = np.random.default_rng(7)
     Wr = rng.normal(0, 1 / np.sqrt(H), (E, H))
     experts = [(rng.normal(0, 1 / np.sqrt(H), (2 * I, H)), rng.normal(0, 1 / np.sqrt(I), (H, I)))
                for _ in range(E + 1)]
+    if fp8:   # W8A8 experts: every weight an e4m3 value times its output row's fp32 scale
+        from oracle import fp8 as ofp8
+
+        def q(w):
+            codes, s = ofp8.quantize_rows(w.astype(np.float32))
+            return codes * s.astype(np.float64)[:, None]
+        experts = [(q(a), q(b)) for a, b in experts]
     return Wr, experts
 
 
-def _worker(rank, world, port, q, tokens=TOKENS):
+def _worker(rank, world, port, q, tokens=TOKENS, fp8=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         from ep_support import OracleRowsBackend
         from oracle import moe
-        Wr, experts = _weights()
+        Wr, experts = _weights(fp8)
         el = E // world
         hidden = torch.from_numpy(np.random.default_rng(100 + rank).normal(0, 1, (tokens[rank], H)))
         backend = OracleRowsBackend(Wr=Wr, bias=None, E=E, k=K, local_experts=experts[rank * el:(rank + 1) * el],
-                                    shared=experts[E])
+                                    shared=experts[E], fp8=fp8)
         ep = ExpertParallelFfn(H=H, E=E, k=K, I=I, T_max=16, backend=backend)
         out = ep.forward(hidden)
         from oracle import comm
@@ -49,33 +56,37 @@ def _worker(rank, world, port, q, tokens=TOKENS):
             q.put((rank, 0.0, 0.0, ep.last_wire, 0))
             return
         idx = moe.route(hidden.numpy(), Wr, None, K)[1]
-        account = comm.element_bytes(idx, H, 8)          # the oracle's per-direction account
+        # the oracle's per-direction element account: float64 rows, or e4m3 codes + a 4-byte scale
+        account = (comm.element_bytes(idx, H, 1) + comm.dispatched_rows(idx) * 4 if fp8
+                   else comm.element_bytes(idx, H, 8))
         ref = moe.forward(hidden.numpy(), Wr, None, lambda e: {"w13": experts[e][0], "w2": experts[e][1]},
-                          E, K, 1)["out"]
+                          E, K, 1, fp8=fp8)["out"]
         q.put((rank, float(np.max(np.abs(out.numpy() - ref))), float(np.max(np.abs(ref))), ep.last_wire, account))
     finally:
         dist.destroy_process_group()
 
 
-def _run(tokens, port):
+def _run(tokens, port, fp8=False):
     world = len(tokens)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q, tokens)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, tokens, fp8)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(180)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
+    row_bytes = H + 4 if fp8 else H * 8                                 # e4m3 + scale, or float64
     for rank, err, scale, wire, account in res:
         assert err <= 1e-12 * max(scale, 1.0), (rank, err)
         # every token sends k rows to the experts' ranks and gets k rows back
         assert wire.tokens == tokens[rank]
-        assert wire.dispatch_sent == tokens[rank] * K * H * 8          # float64 rows in this test
+        assert wire.dispatch_rows == tokens[rank] * K
+        assert wire.dispatch_sent == tokens[rank] * K * row_bytes
         assert wire.dispatch_sent == account                           # = the oracle's element account
-    sent = sum(r[3].dispatch_sent for r in res)
-    back = sum(r[3].combine_sent for r in res)
+    sent = sum(r[3].dispatch_rows for r in res)
+    back = sum(r[3].combine_sent for r in res) // (H * 8)             # float64 rows back
     assert sent == back                                                # the same rows return
 
 
@@ -85,6 +96,16 @@ def test_two_ranks_match_the_single_process_layer():
 
 def test_four_ranks_with_an_empty_and_a_one_token_micro_batch():
     _run({0: 7, 1: 0, 2: 13, 3: 1}, 28600 + os.getpid() % 1000)
+
+
+def test_w8a8_two_ranks_send_e4m3_rows_and_match_the_oracle():
+    # the dispatched rows travel as e4m3 codes with their fp32 scale: H + 4 bytes per row,
+    # the page's FP8 account (A/F 分离, 通信账) plus the scale; outputs equal the oracle's W8A8 layer
+    _run(TOKENS, 21600 + os.getpid() % 1000, fp8=True)
+
+
+def test_w8a8_four_ranks_with_an_empty_micro_batch():
+    _run({0: 5, 1: 11, 2: 0, 3: 3}, 20600 + os.getpid() % 1000, fp8=True)
 
 
 def test_block_tables_regroup_and_restore():
