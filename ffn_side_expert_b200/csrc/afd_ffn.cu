@@ -49,7 +49,6 @@ struct afd_ffn_handle {
   afd_ffn_weights w;
   int device = 0;
   int num_sms = 0;
-  int pair_grid = 0;  // CTAs of the CTA-pair GEMMs: 2 x the pairs that fit on the device at once
   int fused_grid = 0; // CTAs of the fused decode launch (cooperative: all resident at once)
   bool fp8 = false;
   int G = 0;       // E + n_shared
@@ -172,11 +171,10 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false, bool ACT16 = false>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR, ACT16>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              gemm_smem_bytes<BN, ST, SPLIT, MODE, PAIR>());
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, ST, SPLIT, MODE>());
 }
 
 // bf16 large micro-batches with f16 activations: gate/up (f16 act plane) and down (f16 operands)
@@ -207,26 +205,19 @@ constexpr int kAct16BN = 128;
 #ifndef AFD_NB_G2_ST
 #define AFD_NB_G2_ST 5
 #endif
-// AFD_WIDE_PAIR=1 runs each large-micro-batch unit on a CTA pair (2-CTA cluster, M = 256 pair
-// MMAs, N = BN token rows split between the two CTAs): per CTA a 48 KB stage then feeds twice
-// the MMA work of a one-CTA 128 x 128 unit.  Measured on B200 it is slower than one CTA per unit
-// (W8A8 T=8192: 5.04 vs 4.72 ms; bf16 T=4096: 6.03 vs 5.78 ms), so it is off by default.
-#ifndef AFD_WIDE_PAIR
-#define AFD_WIDE_PAIR 0
-#endif
 // bf16 large micro-batch, gate/up
 #ifndef AFD_WB_G1_BN
-#define AFD_WB_G1_BN (AFD_WIDE_PAIR ? 256 : 128)
+#define AFD_WB_G1_BN 128
 #endif
 #ifndef AFD_WB_G1_ST
 #define AFD_WB_G1_ST 4
 #endif
 // bf16 large micro-batch, down (two activation planes per stage)
 #ifndef AFD_WB_G2_BN
-#define AFD_WB_G2_BN (AFD_WIDE_PAIR ? 256 : 128)
+#define AFD_WB_G2_BN 128
 #endif
 #ifndef AFD_WB_G2_ST
-#define AFD_WB_G2_ST (AFD_WIDE_PAIR ? 4 : 3)
+#define AFD_WB_G2_ST 3
 #endif
 // W8A8 decode, gate/up
 #ifndef AFD_NF_G1_BN
@@ -244,17 +235,17 @@ constexpr int kAct16BN = 128;
 #endif
 // W8A8 large micro-batch, gate/up
 #ifndef AFD_WF_G1_BN
-#define AFD_WF_G1_BN (AFD_WIDE_PAIR ? 256 : 128)
+#define AFD_WF_G1_BN 128
 #endif
 #ifndef AFD_WF_G1_ST
 #define AFD_WF_G1_ST 4
 #endif
 // W8A8 large micro-batch, down
 #ifndef AFD_WF_G2_BN
-#define AFD_WF_G2_BN (AFD_WIDE_PAIR ? 256 : 128)
+#define AFD_WF_G2_BN 128
 #endif
 #ifndef AFD_WF_G2_ST
-#define AFD_WF_G2_ST (AFD_WIDE_PAIR ? 6 : 4)
+#define AFD_WF_G2_ST 4
 #endif
 
 // bf16 decode shape: the gate/up and down GEMMs run fused in one launch (MODE 3) with stf ring
@@ -271,58 +262,38 @@ constexpr int kAct16BN = 128;
 #define AFD_WB_F_ST 0
 #endif
 
-template <int BN1, int ST1, int BN2, int ST2, bool SPLIT, int STF = 0, bool PAIR = false>
+template <int BN1, int ST1, int BN2, int ST2, bool SPLIT, int STF = 0>
 struct GemmPairT {
   static constexpr int bn1 = BN1, st1 = ST1, bn2 = BN2, st2 = ST2;
   static constexpr int stf = STF;
   static constexpr bool split = SPLIT;
-  static constexpr bool pair = PAIR;  // both GEMMs on CTA pairs
-  static constexpr bool fused = !PAIR && STF > 0 && BN1 == BN2 && AFD_FUSED;
-  // gate/up units per N tile: 128 gate rows (+ up) per unit, or 256 on a pair
-  static constexpr int gate_rows_per_unit = PAIR ? 256 : 128;
+  static constexpr bool fused = STF > 0 && BN1 == BN2 && AFD_FUSED;
+  static constexpr int gate_rows_per_unit = 128;  // gate/up units: 128 gate rows + 128 up rows
 };
-// Tile shapes: kNarrow (decode), kWide (large micro-batch on CTA pairs when I % 256 == 0) and
-// kWideSingle (large micro-batch, one CTA per unit: any I that is a multiple of 128).
-constexpr int kNarrow = 0, kWide = 1, kWideSingle = 2;
+// Tile shapes: kNarrow (decode micro-batches) and kWide (large micro-batches).
+constexpr int kNarrow = 0, kWide = 1;
 template <bool FP8, int SHAPE>
 struct GemmPair;
 template <>
 struct GemmPair<false, kNarrow>
     : GemmPairT<AFD_NB_G1_BN, AFD_NB_G1_ST, AFD_NB_G2_BN, AFD_NB_G2_ST, true, AFD_NB_F_ST> {};
 template <>
-struct GemmPair<false, kWide>
-    : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true, AFD_WB_F_ST, AFD_WIDE_PAIR> {};
-template <>
-struct GemmPair<false, kWideSingle> : GemmPairT<128, 4, 128, 3, true> {};
+struct GemmPair<false, kWide> : GemmPairT<AFD_WB_G1_BN, AFD_WB_G1_ST, AFD_WB_G2_BN, AFD_WB_G2_ST, true, AFD_WB_F_ST> {};
 template <>
 struct GemmPair<true, kNarrow> : GemmPairT<AFD_NF_G1_BN, AFD_NF_G1_ST, AFD_NF_G2_BN, AFD_NF_G2_ST, false> {};
 template <>
-struct GemmPair<true, kWide>
-    : GemmPairT<AFD_WF_G1_BN, AFD_WF_G1_ST, AFD_WF_G2_BN, AFD_WF_G2_ST, false, 0, AFD_WIDE_PAIR> {};
-template <>
-struct GemmPair<true, kWideSingle> : GemmPairT<128, 4, 128, 4, false> {};
+struct GemmPair<true, kWide> : GemmPairT<AFD_WF_G1_BN, AFD_WF_G1_ST, AFD_WF_G2_BN, AFD_WF_G2_ST, false> {};
 
 // Token-tile TMA box height of the gate/up (gemm = 1) or down (gemm = 2) kernel of a shape.
 template <int SHAPE>
 uint32_t box_rows(bool fp8, int gemm) {
   if (fp8) {
     using P = GemmPair<true, SHAPE>;
-    return gemm == 1 ? GemmShape<P::bn1, false, 0, P::pair>::kBoxRows : GemmShape<P::bn2, false, 1, P::pair>::kBoxRows;
+    return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, false, 1>::kBoxRows;
   }
   using P = GemmPair<false, SHAPE>;
-  return gemm == 1 ? GemmShape<P::bn1, false, 0, P::pair>::kBoxRows
-                   : GemmShape<P::bn2, P::split, 1, P::pair>::kBoxRows;
+  return gemm == 1 ? GemmShape<P::bn1, false, 0>::kBoxRows : GemmShape<P::bn2, P::split, 1>::kBoxRows;
 }
-
-// both wide shapes load token tiles through the same tensor maps, so their boxes must agree
-template <bool FP8>
-constexpr bool wide_boxes_agree() {
-  using A = GemmPair<FP8, kWide>;
-  using B = GemmPair<FP8, kWideSingle>;
-  return GemmShape<A::bn1, false, 0, A::pair>::kBoxRows == GemmShape<B::bn1, false, 0, B::pair>::kBoxRows &&
-         GemmShape<A::bn2, A::split, 1, A::pair>::kBoxRows == GemmShape<B::bn2, B::split, 1, B::pair>::kBoxRows;
-}
-static_assert(wide_boxes_agree<false>() && wide_boxes_agree<true>(), "wide token-tile boxes");
 
 template <bool FP8, int SHAPE>
 cudaError_t set_pair_attrs() {
@@ -330,9 +301,9 @@ cudaError_t set_pair_attrs() {
   if constexpr (P::fused) {
     return set_gemm_attr<P::bn1, (P::fused ? P::stf : 1), FP8, 3, true>();
   } else {
-    cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false, P::pair>();
+    cudaError_t e = set_gemm_attr<P::bn1, P::st1, FP8, 0, false>();
     if (e != cudaSuccess) return e;
-    return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split, P::pair>();
+    return set_gemm_attr<P::bn2, P::st2, FP8, 1, P::split>();
   }
 }
 
@@ -346,37 +317,18 @@ cudaError_t set_all_gemm_attrs() {
   if (e != cudaSuccess) return e;
   e = set_pair_attrs<FP8, kWide>();
   if (e != cudaSuccess) return e;
-  e = set_pair_attrs<FP8, kWideSingle>();
-  if (e != cudaSuccess) return e;
   if constexpr (!FP8) {
-    e = set_gemm_attr<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, false, true>();
+    e = set_gemm_attr<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, true>();
     if (e != cudaSuccess) return e;
-    e = set_gemm_attr<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, false, true>();
+    e = set_gemm_attr<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, true>();
   }
   return e;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool PAIR = false, bool ACT16 = false>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false>
 void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
                  const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
-  if constexpr (PAIR) {
-    // clusters of two CTAs (grid even); the launch error, if any, surfaces through the
-    // cudaGetLastError check that ends the stage
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid & ~1));
-    cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = gemm_smem_bytes<BN, ST, SPLIT, MODE, PAIR>();
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, PAIR>, a, b, a2 ? *a2 : a, b2 ? *b2 : b,
-                       args);
-  } else if constexpr (MODE == 3) {
+  if constexpr (MODE == 3) {
     // the fused kernel's down units wait for act tiles that other CTAs produce, so every CTA of
     // the grid must be resident at once: a cooperative launch guarantees it, or fails (with a
     // launch error that the stage's cudaGetLastError check returns) when it cannot be met
@@ -390,10 +342,10 @@ void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const Gem
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, false, ACT16>, a, b, a2 ? *a2 : a,
+    cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>, a, b, a2 ? *a2 : a,
                        b2 ? *b2 : b, args);
   } else {
-    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, false, ACT16>
+    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>
         <<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
   }
 }
@@ -420,42 +372,6 @@ int fused_grid(int num_sms, int device) {
       return 0;
     }
     return std::min(num_sms, per_sm * num_sms);
-  }
-}
-
-// CTAs of a CTA-pair GEMM launch: every pair of the persistent grid resident at once (two SMs
-// of a TPC each), so no pair waits for another to finish its share of the units.
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT>
-int pair_grid_for(int num_sms) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = gemm_smem_bytes<BN, ST, SPLIT, MODE, true>();
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, true>, &cfg) !=
-          cudaSuccess ||
-      clusters <= 0) {
-    cudaGetLastError();  // clear; fall back to one pair per two SMs
-    return num_sms & ~1;
-  }
-  return std::min(num_sms & ~1, 2 * clusters);
-}
-
-template <bool FP8>
-int pair_grid(int num_sms) {
-  using P = GemmPair<FP8, kWide>;
-  if constexpr (!P::pair) {
-    return num_sms;
-  } else {
-    return std::min(pair_grid_for<P::bn1, P::st1, FP8, 0, false>(num_sms),
-                    pair_grid_for<P::bn2, P::st2, FP8, 1, P::split>(num_sms));
   }
 }
 
@@ -589,13 +505,13 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
     record(h, 7, s);
     return;
   }
-  if constexpr (!FP8 && !NARROW && !P::pair && P::bn1 == kAct16BN && P::bn2 == kAct16BN) {
+  if constexpr (!FP8 && !NARROW && P::bn1 == kAct16BN && P::bn2 == kAct16BN) {
     // (the device schedule was built with P's N tiles, which the f16 kernels share)
     if (h->act16) {  // single-term down GEMM on f16 activations and the f16 copy of W2
       GemmArgs a1 = g1;
       a1.mt_stride = 128;
       record(h, 5, s);
-      launch_gemm<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, false, true>(h->num_sms, h->tm_w13, h->tm_xp[1], a1, s);
+      launch_gemm<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, true>(h->num_sms, h->tm_w13, h->tm_xp[1], a1, s);
       record(h, 6, s);
       GemmArgs a2 = a1;
       a2.unit_base = h->ub2;
@@ -606,13 +522,13 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
       a2.out = h->Y;
       a2.out_ld = c.H;
       record(h, 7, s);
-      launch_gemm<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, false, true>(h->num_sms, h->tm_w2h, h->tm_act16, a2, s);
+      launch_gemm<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, true>(h->num_sms, h->tm_w2h, h->tm_act16, a2, s);
       return;
     }
   }
   record(h, 5, s);
-  const int grid = P::pair ? h->pair_grid : h->num_sms;
-  launch_gemm<P::bn1, P::st1, FP8, 0, false, P::pair>(grid, h->tm_w13, h->tm_xp[shape], g1, s);
+  const int grid = h->num_sms;
+  launch_gemm<P::bn1, P::st1, FP8, 0, false>(grid, h->tm_w13, h->tm_xp[shape], g1, s);
   record(h, 6, s);
   if (FP8)
     quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
@@ -621,19 +537,19 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   g2.K = c.I;
   g2.a_rows = c.H;
   g2.mt_stride = 256;
-  g2.second_off = P::pair ? 0 : 128;  // a pair's down unit is one 256-row tile (128 rows per CTA)
+  g2.second_off = 128;  // a down unit: output rows h.. and h+128..
   g2.out = h->Y;
   g2.out_ld = c.H;
   g2.a_scale = h->w.w2_scale;
   g2.b_scale = h->ascale;
   record(h, 7, s);
-  launch_gemm<P::bn2, P::st2, FP8, 1, P::split, P::pair>(grid, h->tm_w2, h->tm_act[shape], g2, s);
+  launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(grid, h->tm_w2, h->tm_act[shape], g2, s);
 }
 
 int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   const bool narrow = use_narrow(h, T);
-  const int shape = narrow ? kNarrow : (c.I % 256 == 0 ? kWide : kWideSingle);
+  const int shape = narrow ? kNarrow : kWide;
   int bn1, bn2, gate_rows;
   auto pick = [&](auto p) {
     using P = decltype(p);
@@ -643,12 +559,10 @@ int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream
   };
   if (h->fp8) {
     if (shape == kNarrow) pick(GemmPair<true, kNarrow>{});
-    else if (shape == kWide) pick(GemmPair<true, kWide>{});
-    else pick(GemmPair<true, kWideSingle>{});
+    else pick(GemmPair<true, kWide>{});
   } else {
     if (shape == kNarrow) pick(GemmPair<false, kNarrow>{});
-    else if (shape == kWide) pick(GemmPair<false, kWide>{});
-    else pick(GemmPair<false, kWideSingle>{});
+    else pick(GemmPair<false, kWide>{});
   }
   record(h, 4, s);
   build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, bn1, bn2, c.I / gate_rows, c.H / 256,
@@ -656,12 +570,10 @@ int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream
                                           h->err);
   if (h->fp8) {
     if (shape == kNarrow) run_gemms<true, kNarrow>(h, T, s);
-    else if (shape == kWide) run_gemms<true, kWide>(h, T, s);
-    else run_gemms<true, kWideSingle>(h, T, s);
+    else run_gemms<true, kWide>(h, T, s);
   } else {
     if (shape == kNarrow) run_gemms<false, kNarrow>(h, T, s);
-    else if (shape == kWide) run_gemms<false, kWide>(h, T, s);
-    else run_gemms<false, kWideSingle>(h, T, s);
+    else run_gemms<false, kWide>(h, T, s);
   }
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
@@ -876,8 +788,6 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
   if (e != cudaSuccess) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return cuda_fail(nullptr, e); }
-  h->pair_grid = h->fp8 ? pair_grid<true>(h->num_sms) : pair_grid<false>(h->num_sms);
-  if (h->pair_grid < 2) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return AFD_ERR_UNSUPPORTED; }
   h->fused_grid = h->fp8 ? fused_grid<true>(h->num_sms, dev) : fused_grid<false>(h->num_sms, dev);
   if (h->fused_grid < 1) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return AFD_ERR_UNSUPPORTED; }
   router_split_planes_kernel<<<256, 256>>>(weights->router_w, static_cast<size_t>(c.E) * c.H,

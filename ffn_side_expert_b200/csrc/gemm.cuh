@@ -65,7 +65,7 @@ struct GemmArgs {
   int G;                     // groups: routed experts, then the shared expert
   int K;                     // reduction length in elements (H for gate/up and router, I for down)
   int a_rows;                // weight rows per group (2I gate/up, H down); router: valid rows E
-  int mt_stride;             // weight rows between consecutive tile pairs (128 / 256)
+  int mt_stride;             // weight rows between consecutive units' tile pairs (128 gate/up, 256 down)
   int second_off;            // offset of a pair's second tile (I / 128); router: plane stride E
   void* out;                 // MODE 0: act (bf16 planes, or fp32 for W8A8); MODE 1: Y fp32 (bf16 for W8A8);
                              // MODE 2: partial logits fp32 [ksplit][rows][E]
@@ -89,18 +89,14 @@ struct GemmArgs {
   int mt1;                   // gate/up units per N tile (I / 128)
 };
 
-// PAIR: a CTA pair (2-CTA cluster) shares each unit through M = 256 pair MMAs; every CTA holds
-// 128 rows of each weight tile and half of the token tile (BN / 2 rows).  Gate/up units cover
-// 256 gate rows and the 256 matching up rows (two accumulators), down units 256 output rows
-// (one accumulator).
-template <int BN, bool SPLIT_B = false, int MODE = 0, bool PAIR = false>
+template <int BN, bool SPLIT_B = false, int MODE = 0>
 struct GemmShape {
   static constexpr bool kFused = MODE == 3;
-  static constexpr int kNA = MODE == 2 ? 3 : (PAIR && MODE == 1 ? 1 : 2);   // weight tiles per stage
-  static constexpr int kNDU = MODE == 2 ? 1 : (PAIR && MODE == 1 ? 1 : 2);  // accumulators per unit
+  static constexpr int kNA = MODE == 2 ? 3 : 2;   // weight tiles per stage
+  static constexpr int kNDU = MODE == 2 ? 1 : 2;  // accumulators per unit
   static constexpr int kATile = 128 * 128;              // one 128-row x 128-byte weight tile
   static constexpr int kAStage = kNA * kATile;
-  static constexpr int kBRows = PAIR ? BN / 2 : BN;     // token rows of this CTA's tile
+  static constexpr int kBRows = BN;                     // token rows of a tile
   static constexpr int kBTile = kBRows * 128;           // up to kBRows token rows x 128 bytes
   static constexpr int kBStage = (SPLIT_B ? 2 : 1) * kBTile;
   static constexpr int kStageBytes = kAStage + kBStage;
@@ -124,7 +120,6 @@ struct GemmShape {
                                    : kColsUsed <= 256 ? 256 : 512;
   static_assert(kColsUsed <= 512, "TMEM has 512 columns");
   static_assert(BN % 16 == 0 && BN <= 256, "N tile");
-  static_assert(!PAIR || ((MODE == 0 || MODE == 1) && !kConcat), "pairs serve the wide gate/up and down GEMMs");
   static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 };
 
@@ -133,10 +128,10 @@ struct GemmShape {
 constexpr int kMaxGroups = 257;
 constexpr int kSchedBytes = (kMaxGroups + 1) * 16;
 
-template <int BN, int STAGES, bool SPLIT_B, int MODE = 0, bool PAIR = false>
+template <int BN, int STAGES, bool SPLIT_B, int MODE = 0>
 constexpr int gemm_smem_bytes() {
   return (MODE == 3 ? 2 : 1) * kSchedBytes + 1024 /*alignment slack*/ +
-         STAGES * GemmShape<BN, SPLIT_B, MODE, PAIR>::kStageBytes + 256 /*barriers*/;
+         STAGES * GemmShape<BN, SPLIT_B, MODE>::kStageBytes + 256 /*barriers*/;
 }
 
 // Largest g with tab[g].x (first unit of group g) <= u; the table sits in shared memory.
@@ -235,15 +230,15 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
 // f16 operands) -- f16 keeps 10 mantissa bits where bf16 keeps 7, so one term suffices.  Each
 // token row is stored divided by its power-of-two scale b_scale[row] (f16_row_scale: the row's
 // bound on |act| stays inside the f16 range), and the down epilogue multiplies it back.
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool PAIR = false, bool ACT16 = false>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool ACT16 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs args) {
   static_assert(!(SPLIT_B && (FP8 || (MODE != 1 && MODE != 3))), "two-term B only for the bf16 down GEMM");
   static_assert(!((MODE == 2 || MODE == 3) && FP8), "router and fused modes run on bf16");
-  static_assert(!ACT16 || (!FP8 && !SPLIT_B && !PAIR && (MODE == 0 || MODE == 1)), "f16 activations: wide bf16 GEMMs");
-  using S = GemmShape<BN, SPLIT_B, MODE, PAIR>;
+  static_assert(!ACT16 || (!FP8 && !SPLIT_B && (MODE == 0 || MODE == 1)), "f16 activations: wide bf16 GEMMs");
+  using S = GemmShape<BN, SPLIT_B, MODE>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
 
@@ -268,11 +263,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // CTA pair: rank in the pair, the pair's index and count; the unit loop runs over pairs
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  const bool leader = rank == 0;
+  const int unit0 = static_cast<int>(blockIdx.x);
+  const int unit_step = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -281,7 +273,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int i = 0; i < kNacc; ++i) {
       mbar_init(tfull + 8u * i, 1);
-      mbar_init(tempty + 8u * i, (PAIR ? 2 : 1) * kEpiWarps);
+      mbar_init(tempty + 8u * i, kEpiWarps);
     }
     mbar_init(done_bar, 1);
     for (int i = 0; i < kNacc; ++i) mbar_init(epi_bar + 8u * i, kEpiWarps);
@@ -295,13 +287,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   }
   if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(smem_u32(tmem_slot), S::kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
+    tmem_relinquish();
   }
   if (args.single_rows < 0) {
     for (int g = threadIdx.x; g <= args.G; g += blockDim.x) {
@@ -316,8 +303,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
   tc_fence_before();
   __syncthreads();
-  // the peer's barriers are initialised before any TMA or commit of the pair reaches them
-  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -332,25 +317,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t ph = 0;
     int issued = 0;
     bool ok = true;
-    // a pair's stages complete on the first CTA's full barriers (both halves counted there)
-    const uint32_t full_tx = PAIR ? mapa_shared(full, 0) : full;
     for (int u = unit0; u < total && ok; u += unit_step) {
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       // the down side of the fused kernel uses the second set of maps and coordinates
       const bool down = MODE == 3 && w.mode == 1;
       const CUtensorMap* mA = down ? &tmA2 : &tmA;
       const CUtensorMap* mB = down ? &tmB2 : &tmB;
-      const int ya = (down ? w.g * args.a_rows2 + w.mt * args.mt_stride2 : w.g * args.a_rows + w.mt * args.mt_stride) +
-                     (PAIR ? 128 * static_cast<int>(rank) : 0);
+      const int ya = down ? w.g * args.a_rows2 + w.mt * args.mt_stride2 : w.g * args.a_rows + w.mt * args.mt_stride;
       const int soff = down ? args.second_off2 : args.second_off;
       const bool two = SPLIT_B && (MODE != 3 || down);           // hi and lo planes
       const int boxr = (MODE == 3 && !down) ? S::kBoxRowsX : S::kBoxRows;
-      // this CTA's token rows: all n16 rows, or its half of them in a pair
-      const int brows = PAIR ? w.n16 / 2 : w.n16;
-      const int brow0 = w.row0 + (PAIR ? static_cast<int>(rank) * brows : 0);
+      const int brows = w.n16;  // token rows loaded (the MMA reads n16 of them)
+      const int brow0 = w.row0;
       const int nbox = (brows + boxr - 1) / boxr;                  // token-tile boxes per plane
-      const uint32_t tx = (PAIR ? 2u : 1u) *
-                          (S::kAStage + (two ? 2u : 1u) * static_cast<uint32_t>(nbox * boxr) * 128u);
+      const uint32_t tx = S::kAStage + (two ? 2u : 1u) * static_cast<uint32_t>(nbox * boxr) * 128u;
       // the lo activation rows follow the (padded) hi rows or sit one tile further
       const uint32_t lo_off = S::kConcat ? static_cast<uint32_t>(S::npad(w.n16)) * 128u : S::kBTile;
       const uint64_t apol = MODE == 2 ? kEvictLast : args.a_policy;
@@ -358,43 +338,31 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int kc = w.kc0; kc < w.kc1; ++kc) {
         if (!mbar_wait(empty + 8u * s, ph ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t st = base + s * S::kStageBytes;
-        const uint32_t fb = full_tx + 8u * s;
+        const uint32_t fb = full + 8u * s;
         const int x = kc * kKChunk;
-        if (leader) mbar_arrive_expect_tx(full + 8u * s, tx);
-        // the tile pair (MODE 0/1), one tile (pair down), or the three router planes (MODE 2)
+        mbar_arrive_expect_tx(full + 8u * s, tx);
+        // the tile pair (MODE 0/1) or the three router planes (MODE 2)
 #pragma unroll
-        for (int i = 0; i < S::kNA; ++i) {
-          if constexpr (PAIR) tma_load_2d_pair(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
-          else tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
-        }
+        for (int i = 0; i < S::kNA; ++i) tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
         const uint32_t sb = st + S::kAStage;
-        for (int b = 0; b < nbox; ++b) {
-          if constexpr (PAIR) tma_load_2d_pair(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
-          else tma_load_2d(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
-        }
+        for (int b = 0; b < nbox; ++b) tma_load_2d(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
         if (two) {
-          for (int b = 0; b < nbox; ++b) {
-            const int y = args.lo_rows + brow0 + b * boxr;
-            if constexpr (PAIR) tma_load_2d_pair(sb + lo_off + b * boxr * 128, mB, fb, x, y, kEvictLast);
-            else tma_load_2d(sb + lo_off + b * boxr * 128, mB, fb, x, y, kEvictLast);
-          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sb + lo_off + b * boxr * 128, mB, fb, x, args.lo_rows + brow0 + b * boxr, kEvictLast);
         }
         ++issued;
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
     if (!ok) { *abort_flag = 1; atomicOr(args.err, kErrTimeout); }
-    // drain: the last min(issued, STAGES) stages may still be landing in shared memory.  The
-    // second CTA of a pair cannot see its loads land (they count on the first CTA's barrier);
-    // it waits until the pair's MMAs have consumed them instead (bounded either way).
+    // drain: the last min(issued, STAGES) stages may still be landing in shared memory (bounded)
     for (int i = 0; i < min(issued, STAGES); ++i) {
       if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
       volatile int never = 0;
-      mbar_wait((leader ? full : empty) + 8u * s, ph, &never);
+      mbar_wait(full + 8u * s, ph, &never);
     }
-  } else if (warp == 1 && lane == 0 && leader) {
+  } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
-    // (in a pair, the first CTA issues the pair's MMAs; its commits reach both CTAs)
     int s = 0;
     uint32_t ph = 0;
     int acc = 0;
@@ -404,11 +372,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
       const bool cat = S::kConcat && down;
-      const uint32_t idesc = idesc_mn(PAIR ? 256 : 128, cat ? 2 * S::npad(w.n16) : w.n16, FP8, ACT16 && MODE == 1);
-      // (a pair's accumulators are released by the epilogue warps of both CTAs)
-      const bool freed = PAIR ? mbar_wait_cluster(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)
-                              : mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag);
-      if (!freed) { ok = false; break; }
+      const uint32_t idesc = idesc_mn(128, cat ? 2 * S::npad(w.n16) : w.n16, FP8, ACT16 && MODE == 1);
+      if (!mbar_wait(tempty + 8u * acc, acc_ph ^ 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d0 = tmem + static_cast<uint32_t>(acc * S::kUnitCols);
       const uint32_t d1 = d0 + S::kUnitCols / 2;
@@ -427,14 +392,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_mma<false>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             tc_mma<false>(d0, da1 + 2 * kk, db + 2 * kk, idesc, 1u);
             tc_mma<false>(d0, da2 + 2 * kk, db + 2 * kk, idesc, 1u);
-          } else if constexpr (PAIR) {
-            // gate/up: the 256 gate rows and the 256 up rows; down: 256 output rows (+ lo plane)
-            tc_mma_pair<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-            if constexpr (S::kNDU == 2) tc_mma_pair<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
-            if constexpr (SPLIT_B) {
-              const uint64_t dl = sw128_desc(st + S::kAStage + S::kBTile);
-              tc_mma_pair<FP8>(d0, da0 + 2 * kk, dl + 2 * kk, idesc, 1u);
-            }
           } else {
             tc_mma<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
             tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
@@ -447,20 +404,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
           }
         }
-        // frees the stage (in both CTAs of a pair) once these MMAs have read it
-        if constexpr (PAIR) tc_commit_pair_mc(empty + 8u * s, 0x3);
-        else tc_commit(empty + 8u * s);
+        tc_commit(empty + 8u * s);  // frees the stage once these MMAs have read it
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
-      if constexpr (PAIR) tc_commit_pair_mc(tfull + 8u * acc, 0x3);
-      else tc_commit(tfull + 8u * acc);
+      tc_commit(tfull + 8u * acc);
       if (++acc == kNacc) { acc = 0; acc_ph ^= 1u; }
     }
     if (!ok) { *abort_flag = 1; atomicOr(args.err, kErrTimeout); }
     // every MMA issued above has completed once this commit arrives
-    if constexpr (PAIR) tc_commit_pair(done_bar);
-    else tc_commit(done_bar);
+    tc_commit(done_bar);
     volatile int never = 0;
     mbar_wait(done_bar, 0, &never);
   } else if (warp >= 2 && warp < 2 + kEpiWarps) {
@@ -472,8 +425,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     int acc = 0;
     uint32_t acc_ph = 0;
     uint32_t epi_ph = 0;  // parity bit per accumulator buffer
-    // a pair's epilogue warps release an accumulator on the first CTA's barrier
-    const uint32_t tempty_rel = PAIR ? mapa_shared(tempty, 0) : tempty;
     for (int u = unit0; u < total; u += unit_step) {
       const Unit w = decode_unit<BN, MODE>(args, sched, sched2, u, kchunks, kchunks2);
       if (!mbar_wait(tfull + 8u * acc, acc_ph, abort_flag)) {
@@ -487,7 +438,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // weight rows of this thread in the two tiles
       const bool down = MODE == 1 || (MODE == 3 && w.mode == 1);
       const int wrow0 = w.mt * (MODE == 3 && down ? args.mt_stride2 : args.mt_stride) +
-                        (PAIR ? 128 * static_cast<int>(rank) : 0) + m;
+                        m;
       const int wrow1 = wrow0 + (MODE == 3 && down ? args.second_off2 : args.second_off);
       if constexpr (MODE == 2) {  // partial logits [split][t][e]; rows past E are padding
         const int e = wrow0;
@@ -602,8 +553,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
       }
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(tempty_rel + 8u * acc);
-        else mbar_arrive(tempty + 8u * acc);
+        mbar_arrive(tempty + 8u * acc);
       }
       if (++acc == kNacc) { acc = 0; acc_ph ^= 1u; }
     }
@@ -611,12 +561,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   tc_fence_before();
   __syncthreads();
-  // neither CTA of a pair leaves while the other may still signal its barriers
-  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    if constexpr (PAIR) tmem_dealloc_pair(tmem, S::kTmemCols);
-    else tmem_dealloc(tmem, S::kTmemCols);
+    tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 

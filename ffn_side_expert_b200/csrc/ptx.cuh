@@ -65,19 +65,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with acquire at cluster scope: for barriers that other CTAs of the cluster arrive on.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(static_cast<uint32_t>(AFD_SUSPEND_NS > 0 ? AFD_SUSPEND_NS : 1000))
-      : "memory");
-  return ok != 0;
-}
-
 // About 2 s of SM clock: far above any legitimate wait of one tile, far below a watchdog.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
@@ -88,17 +75,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
-  }
-}
-
-// mbar_wait for a barrier that other CTAs of the cluster arrive on (acquire at cluster scope).
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
@@ -125,92 +101,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// ------------------------------------------------------------------ CTA pairs (2-CTA clusters)
-// Rank of this CTA in its cluster.
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// All threads of all CTAs of the cluster: release this CTA's prior writes, acquire the others'.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Shared-memory address `a` of this CTA mapped to the same offset in the cluster CTA `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
-  uint32_t d;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(rank));
-  return d;
-}
-
-// Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared), releasing
-// this thread's prior memory operations at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-
-// TMA tile load of a CTA pair: the box lands in this CTA's shared memory at `dst` and its bytes
-// are counted on the mbarrier at `cluster_bar`, which may be the peer CTA's (the pair's MMAs are
-// issued by one CTA, which waits for both halves on its own barrier).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t cluster_bar,
-                                                 int32_t x, int32_t y, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
-// TMEM allocation shared by a CTA pair: one warp of each CTA (the same warp index in both) issues
-// it with the same destination offset; both CTAs get the same TMEM address.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Pair MMA (issued by the pair's first CTA): M = 256, rows 0..127 of A and of D in CTA 0, rows
-// 128..255 in CTA 1; B's N rows split in halves the same way; both CTAs' operands at the same
-// shared-memory offsets.
-template <bool kFp8>
-__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  if constexpr (kFp8) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem), "l"(adesc),
-        "l"(bdesc), "r"(idesc), "r"(accumulate));
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem), "l"(adesc),
-        "l"(bdesc), "r"(idesc), "r"(accumulate));
-  }
-}
-
-// Arrive once on the mbarrier at offset `bar` of every CTA in `cta_mask` when the pair MMAs
-// issued so far by this thread have completed.
-__device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-               "h"(cta_mask)
-               : "memory");
-}
-
-// Arrive once on this CTA's mbarrier `bar` when the pair MMAs issued so far have completed.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)
@@ -272,8 +163,7 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
   }
 }
 
-// Instruction descriptor: fp32 accumulator, A and B K-major, M = m (128, or 256 for a CTA
-// pair), N = n (multiple of 16).  Operand format (A and B alike): bf16 or f16 (kind::f16: 1 =
+// Instruction descriptor: fp32 accumulator, A and B K-major, M = m (128), N = n (multiple of 16).  Operand format (A and B alike): bf16 or f16 (kind::f16: 1 =
 // bf16, 0 = f16) or e4m3 (kind::f8f6f4: 0).
 __host__ __device__ constexpr uint32_t idesc_mn(int m, int n, bool fp8, bool f16 = false) {
   return (1u << 4)                                             // D format f32

@@ -127,9 +127,9 @@ def test_all_experts_selected_with_shared_expert():
 
 @pytest.mark.parametrize("T", [600, 520])
 def test_wide_tiles_with_several_n_tiles_per_expert(T):
-    # T*k > 32 E selects the wide tiles: N tiles of up to 256 rows, each split between the two
-    # CTAs of a pair.  ~T/2 rows per expert gives several N tiles with a ragged last one; the
-    # shared expert's T rows end in a 88-row tile (T=600) or a 16-row one, 8 rows per CTA (T=520)
+    # T*k > 32 E selects the wide tiles: N tiles of up to 128 rows.  ~T/2 rows per expert gives
+    # several N tiles with a ragged last one; the shared expert's T rows end in an 88-row tile
+    # (T=600) or an 8-row one (T=520)
     cfg = synth.MoEConfig("wide", T=600, H=256, E=2, k=1, I=256, S=1, seed=24)
     L = Layer(cfg, redraws=_redraws(cfg))
     try:
@@ -139,9 +139,8 @@ def test_wide_tiles_with_several_n_tiles_per_expert(T):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp8"])
-def test_wide_tiles_single_cta_when_i_is_not_a_multiple_of_256(dtype):
-    # I = 384 = 3 x 128: gate/up units of 256 rows cannot tile it, so the wide shape runs the
-    # one-CTA kernels (128-row units, N tiles of 128)
+def test_wide_tiles_when_i_is_not_a_multiple_of_256(dtype):
+    # I = 384 = 3 x 128: an odd number of 128-row gate/up units per N tile (wide tiles, N <= 128)
     cfg = synth.MoEConfig("wide384", T=300, H=256, E=2, k=1, I=384, S=1, dtype=dtype, seed=27)
     L = Layer(cfg, redraws=_redraws(cfg))
     try:
