@@ -117,7 +117,8 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 20 ms; only the samples written while
+    the timed region runs (between entering and leaving the context) are summarised."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -126,20 +127,31 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.f = None
+        self.first = self.last = 0
+
+    def _lines(self) -> list:
+        self.f.flush()
+        with open(self.f.name) as fh:
+            return [r for r in fh.read().splitlines() if r.count(",") >= 8]
 
     def __enter__(self):
         try:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
-        time.sleep(0.3)
+        if self.proc is not None:
+            t_end = time.monotonic() + 3.0        # wait until the sampler is producing lines
+            while time.monotonic() < t_end and not self._lines():
+                time.sleep(0.02)
+            self.first = len(self._lines())
         return self
 
     def __exit__(self, *a):
         if self.proc is not None:
+            self.last = len(self._lines())
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -149,24 +161,27 @@ class ClockSampler:
     def summary(self) -> dict:
         if self.proc is None or self.f is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.f.flush()
-        with open(self.f.name) as fh:
-            rows = [r.split(",") for r in fh.read().strip().splitlines() if r.count(",") >= 8]
+        lines = self._lines()
         os.unlink(self.f.name)
-        sm, smax, reasons = [], None, set()
+        # samples written during the timed region; the one just before it when the region is
+        # shorter than the sampling period
+        window = lines[self.first:self.last] if self.last > self.first else lines[max(0, self.first - 1):self.first]
+        rows = [r.split(",") for r in window]
+        sm, smax, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
                 sm.append(float(r[1]))
                 smax = float(r[2])
+                power.append(float(r[3]))
             except ValueError:
                 continue
             for nm, v in zip(names, r[5:9]):
                 if v.strip().lower() == "active":
                     reasons.add(nm)
-        busy = [s for s in sm if smax and s > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "sm_mhz_min": min(sm) if sm else None, "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm), "period_ms": 20}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -409,12 +424,10 @@ def fused_decode(cfg) -> bool:
 
 
 def launches_per_step(cfg) -> int:
-    """Library kernel launches of one forward: router GEMM, selection (top-k + refined weights),
+    """Library kernel launches of one forward: router GEMM, top-k selection and gate weights,
     dispatch count, dispatch scan, gather, schedule, then the fused expert kernel (bf16 decode
-    shape) or gate/up GEMM (+ W8A8 activation quantisation) and down GEMM, then combine; from
-    T = 2048 selection and refinement are two launches."""
-    n = 8 if fused_decode(cfg) else (10 if cfg.dtype == "fp8" else 9)
-    return n + (1 if cfg.T >= 2048 else 0)
+    shape) or gate/up GEMM (+ W8A8 activation quantisation) and down GEMM, then combine."""
+    return 8 if fused_decode(cfg) else (10 if cfg.dtype == "fp8" else 9)
 
 
 def rooflines(cfg, acct, ms, kernel_ms, traffic=None):

@@ -37,8 +37,12 @@ namespace {
 // rows in 64-row boxes, so they share one tensor map.
 constexpr int kRouterBN = 64, kRouterStages = 3;
 constexpr int kRouterBNWide = 128, kRouterWideT = 1024;
-// Below this micro-batch size the top-k selection and the weight refinement run as one launch.
-constexpr int kSelectFusedMaxT = 2048;
+// Longest stretch of H (in 64-element chunks) one tensor-core accumulation of the router covers:
+// the partial logits of consecutive stretches are then added in fp32, in order, by the top-k
+// kernel.  Measured on B200 at the DeepSeek-V3 router shape, the gate weights from the summed
+// logits stay within 7e-7 of the fp64 ones with 384-element stretches but drift to 9e-6 with a
+// single 3584-element one; 1024 elements keeps the accumulations short at every micro-batch size.
+constexpr int kRouterMaxSplitChunks = 16;
 
 thread_local int g_create_cuda_error = 0;
 
@@ -375,11 +379,13 @@ int fused_grid(int num_sms, int device) {
   }
 }
 
-// K split of the tensor-core router: enough units to cover the SMs, every split non-empty.
+// K split of the tensor-core router: enough units to cover the SMs and stretches of at most
+// kRouterMaxSplitChunks chunks, every split non-empty.
 void router_ksplit(int T, int H, int E, int sms, int bn, int* ksplit, int* kc_per) {
   const int kchunks = H / 64;
   const int base = ((T + bn - 1) / bn) * ((E + 127) / 128);
-  const int want = std::max(1, std::min(kchunks, (sms + base - 1) / base));
+  const int min_split = (kchunks + kRouterMaxSplitChunks - 1) / kRouterMaxSplitChunks;
+  const int want = std::max(min_split, std::min(kchunks, (sms + base - 1) / base));
   *kc_per = (kchunks + want - 1) / want;
   *ksplit = (kchunks + *kc_per - 1) / *kc_per;
 }
@@ -422,21 +428,9 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
   else
     launch_gemm<kRouterBN, kRouterStages, false, 2, false>(std::min(h->num_sms, a.single_total), h->tm_wr, tm_h, a, s);
   record(h, 1, s);
+  // selection and gate weights from the summed partial logits, a warp per token
   const float* bias = c.has_router_bias ? h->w.router_bias : nullptr;
-  if (T < kSelectFusedMaxT) {
-    // small micro-batches: selection and refinement in one launch, up to four warps per selected
-    // expert splitting the dot product (few CTAs, so each one's chain of loads is the latency)
-    const int slices = std::max(1, std::min(4, 32 / c.k));
-    const int threads = std::max(256, 32 * c.k * slices);
-    router_select_kernel<<<T, threads, 0, s>>>(h->part, ksplit, bias, static_cast<const __nv_bfloat16*>(hidden),
-                                               h->w.router_w, T, c.E, c.H, c.k, idx, w);
-  } else {
-    // large ones: a warp per token selects, then a CTA per token refines (measured faster there
-    // than the one-launch form, whose warps wait on the selection)
-    router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
-    router_refine_kernel<<<T, 32 * c.k, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), h->w.router_w, bias,
-                                               c.H, c.k, idx, w);
-  }
+  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }

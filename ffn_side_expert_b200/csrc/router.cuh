@@ -7,10 +7,9 @@
 // order (ties to the lower expert), w = softmax over the selected logits.
 //
 // The handle's router (afd_ffn_route / afd_ffn_forward) is MODE 2 of the grouped GEMM in
-// gemm.cuh (tensor cores, Wr as three bf16 planes, split-K partial logits) followed by
-// router_select_kernel (selection + exact fp32 refinement of the k selected logits + softmax,
-// one CTA per token) for small micro-batches, router_topk_kernel + router_refine_kernel for
-// large ones (a warp per token for the selection, a CTA per token for the refinement).
+// gemm.cuh (tensor cores, Wr as three bf16 planes whose sum represents it to ~2^-27, split-K
+// partial logits over stretches of at most 1024 elements of H) followed by router_topk_kernel,
+// which adds the partials in split order in fp32 and selects and normalises from those logits.
 // The allocation-free afd_ffn_route_static uses router_logits_kernel (fp32 FMA GEMM, 64 tokens
 // x 64 experts per CTA, 4x4 outputs per thread, K tiles of 32 in shared memory, optionally split
 // over K) and router_topk_kernel (one warp per token; 8 logits per lane, k rounds of warp
@@ -151,159 +150,6 @@ router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __re
   if (lane < k) {
     idx[static_cast<size_t>(t) * k + lane] = my_e;
     w[static_cast<size_t>(t) * k + lane] = z / sum;
-  }
-}
-
-// Gate weights from exact fp32 logits of the selected experts.  The tensor-core router's fp32
-// accumulation over 3 x H terms is a few bits short of an fp32 FMA chain: good enough to select
-// (the selection margin is far larger), not for the weights.  One CTA per token, warp j
-// recomputes logit j = hidden[t] . Wr[idx[t][j]] (+ bias) with fp32 FMAs (each lane takes 8
-// consecutive hidden values per step, the warp adds the lane sums); warp 0 then writes the
-// softmax over the k logits.  blockDim = 32 * k.
-__global__ void __launch_bounds__(1024)
-router_refine_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr,
-                     const float* __restrict__ bias, int H, int k, const int32_t* __restrict__ idx,
-                     float* __restrict__ w) {
-  __shared__ float lg[32];
-  const int t = blockIdx.x;
-  const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = idx[static_cast<size_t>(t) * k + j];
-  float acc = 0.f;
-  if (e >= 0) {
-    const uint4* hr = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H);
-    const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
-#pragma unroll 4
-    for (int c = lane; c < H / 8; c += 32) {
-      const uint4 hv = hr[c];
-      const float4 w0 = wrow[2 * c], w1 = wrow[2 * c + 1];
-      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hv);
-      float2 f;
-      f = __bfloat1622float2(b[0]); acc = fmaf(f.x, w0.x, acc); acc = fmaf(f.y, w0.y, acc);
-      f = __bfloat1622float2(b[1]); acc = fmaf(f.x, w0.z, acc); acc = fmaf(f.y, w0.w, acc);
-      f = __bfloat1622float2(b[2]); acc = fmaf(f.x, w1.x, acc); acc = fmaf(f.y, w1.y, acc);
-      f = __bfloat1622float2(b[3]); acc = fmaf(f.x, w1.z, acc); acc = fmaf(f.y, w1.w, acc);
-    }
-    acc = warp_sum(acc);
-    if (bias) acc += bias[e];
-  } else {
-    acc = -INFINITY;
-  }
-  if (lane == 0) lg[j] = acc;
-  __syncthreads();
-  if (j == 0) {
-    const float v = lane < k ? lg[lane] : -INFINITY;
-    const float vmax = __shfl_sync(0xffffffffu, v, 0);  // selection order: logit 0 is the largest
-    const float z = lane < k ? expf(v - vmax) : 0.f;
-    const float sum = warp_sum(z);
-    if (lane < k) w[static_cast<size_t>(t) * k + lane] = z / sum;
-  }
-}
-
-// Selection and gate weights in one launch, one CTA per token (blockDim = max(256, 32 k)):
-//  1. thread e sums expert e's partial logits in split order (+ bias) into shared memory -- the
-//     same additions, in the same order, as router_topk_kernel, so the selection is identical;
-//  2. warp 0 picks the k largest (descending, ties to the lower index), as router_topk_kernel;
-//  3. the warps split the k exact fp32 dot products hidden[t] . Wr[idx[t][j]]: warp w works on
-//     selection j = w % k over the H slice (w / k) of (warps / k) slices; the slice sums are
-//     added in slice order (+ bias);
-//  4. warp 0 writes the softmax over the k refined logits.
-constexpr int kSelectMaxThreads = 1024;
-__global__ void __launch_bounds__(kSelectMaxThreads)
-router_select_kernel(const float* __restrict__ part, int nsplit, const float* __restrict__ bias,
-                     const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ wr, int T, int E, int H,
-                     int k, int32_t* __restrict__ idx, float* __restrict__ w) {
-  __shared__ float lg[256];
-  __shared__ int sel[32];
-  __shared__ float slice_sum[32][32];  // [slice][selection]
-  const int t = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
-  for (int e = tid; e < 256; e += blockDim.x) {
-    float v = -INFINITY;
-    if (e < E) {
-      v = 0.f;
-      const float* pe = part + static_cast<size_t>(t) * E + e;
-      const size_t plane = static_cast<size_t>(T) * E;
-#pragma unroll 4
-      for (int sp = 0; sp < nsplit; ++sp) v += pe[sp * plane];
-      if (bias) v += bias[e];
-    }
-    lg[e] = v;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float v[8];
-    unsigned taken = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = lg[lane + 32 * i];
-    int my_e = -1;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {  // expert index grows with i: the first best is the lowest
-        const int e = lane + 32 * i;
-        if (e < E && !(taken >> i & 1u) && (v[i] > bv || (be == 0x7fffffff && v[i] == bv))) {
-          bv = v[i];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == j) my_e = (be == 0x7fffffff) ? -1 : be;
-    }
-    if (lane < k) {
-      sel[lane] = my_e;
-      idx[static_cast<size_t>(t) * k + lane] = my_e;
-    }
-  }
-  __syncthreads();
-  const int slices = nwarps / k;  // >= 1: blockDim >= 32 k
-  if (warp < slices * k) {
-    const int j = warp % k, sl = warp / k;
-    const int e = sel[j];
-    float acc = 0.f;
-    if (e >= 0) {
-      const int chunks = H / 8;  // 8 hidden values per 16-byte load
-      const int c0 = static_cast<int>((static_cast<long long>(chunks) * sl) / slices);
-      const int c1 = static_cast<int>((static_cast<long long>(chunks) * (sl + 1)) / slices);
-      const uint4* hr = reinterpret_cast<const uint4*>(hidden + static_cast<size_t>(t) * H);
-      const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(e) * H);
-#pragma unroll 4
-      for (int c = c0 + lane; c < c1; c += 32) {
-        const uint4 hv = hr[c];
-        const float4 w0 = wrow[2 * c], w1 = wrow[2 * c + 1];
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hv);
-        float2 f;
-        f = __bfloat1622float2(b[0]); acc = fmaf(f.x, w0.x, acc); acc = fmaf(f.y, w0.y, acc);
-        f = __bfloat1622float2(b[1]); acc = fmaf(f.x, w0.z, acc); acc = fmaf(f.y, w0.w, acc);
-        f = __bfloat1622float2(b[2]); acc = fmaf(f.x, w1.x, acc); acc = fmaf(f.y, w1.y, acc);
-        f = __bfloat1622float2(b[3]); acc = fmaf(f.x, w1.z, acc); acc = fmaf(f.y, w1.w, acc);
-      }
-      acc = warp_sum(acc);
-    }
-    if (lane == 0) slice_sum[sl][j] = acc;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float v = -INFINITY;
-    if (lane < k) {
-      const int e = sel[lane];
-      if (e >= 0) {
-        v = 0.f;
-        for (int sl = 0; sl < slices; ++sl) v += slice_sum[sl][lane];
-        if (bias) v += bias[e];
-      }
-    }
-    const float vmax = __shfl_sync(0xffffffffu, v, 0);  // selection order: logit 0 is the largest
-    const float z = lane < k ? expf(v - vmax) : 0.f;
-    const float sum = warp_sum(z);
-    if (lane < k) w[static_cast<size_t>(t) * k + lane] = z / sum;
   }
 }
 

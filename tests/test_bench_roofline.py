@@ -31,7 +31,7 @@ def test_w8a8_large_chunk_gate_up_is_tensor_bound():
     assert roof["algorithmic_flops_per_launch"] == 4 * cfg.H * cfg.I * rows
     assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
     assert roof["peak"] == 2 * bench.load_peaks()[0]["bf16_tflops"]         # e4m3 = 2 x bf16
-    assert bench.launches_per_step(cfg) == 11                             # T >= 2048: +1
+    assert bench.launches_per_step(cfg) == 10
 
 
 def test_bf16_large_micro_batch_gate_up_is_hbm_bound():
@@ -39,4 +39,27 @@ def test_bf16_large_micro_batch_gate_up_is_hbm_bound():
     roof, _ = bench.rooflines(cfg, acct, ms=5.0, kernel_ms=2.7)
     assert roof["bound"] == "hbm"
     assert roof["algorithmic_bytes_per_launch"] == 257 * 2 * 2048 * 7168 * 2
-    assert bench.launches_per_step(cfg) == 10
+    assert bench.launches_per_step(cfg) == 9
+
+
+def test_clock_summary_keeps_only_the_timed_window(tmp_path):
+    # lines written before the region (the sampler warming up) and after it are left out; the
+    # last line before the region stands in when the region is shorter than one period
+    import os
+    f = open(tmp_path / "clk.csv", "w+")
+    idle = "0, 1965, 1965, 200.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    load = "0, 1320, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active"
+    f.write("\n".join([idle] * 10 + [load] * 3 + [idle] * 4) + "\n")
+    f.flush()
+    c = bench.ClockSampler(0)
+    c.f, c.proc, c.first, c.last = f, object(), 10, 13
+    s = c.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1320.0 and s["sm_mhz_min"] == 1320.0
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 995.0
+    assert not os.path.exists(tmp_path / "clk.csv")
+    f = open(tmp_path / "clk2.csv", "w+")
+    f.write("\n".join([idle] * 5 + [load]) + "\n")
+    f.flush()
+    c.f, c.first, c.last = f, 6, 6                           # no sample inside a short region
+    s2 = c.summary()
+    assert s2["samples"] == 1 and s2["sm_mhz"] == 1320.0

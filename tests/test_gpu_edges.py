@@ -151,8 +151,8 @@ def test_wide_tiles_when_i_is_not_a_multiple_of_256(dtype):
 
 @pytest.mark.parametrize("T", [1500, 2100])
 def test_router_tiles_around_the_size_thresholds(T):
-    # T >= 1024: 128-token router GEMM tiles; T < 2048: selection and refinement in one launch,
-    # T >= 2048: separate selection and refinement kernels
+    # T >= 1024: 128-token router GEMM tiles (T = 1500, 2100), against 64-token tiles below;
+    # with H = 256 every micro-batch size keeps the reduction in one stretch of H
     cfg = synth.MoEConfig("thresholds", T=2100, H=256, E=16, k=4, I=256, S=1, seed=29)
     L = Layer(cfg, redraws=_redraws(cfg))
     try:
