@@ -10,6 +10,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace afd {
@@ -23,6 +25,12 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p, size_t i) {
 }
 
 // Ys: the shared expert's rows [T][H], or nullptr when they follow the routed rows in Y.
+// Grid: (T, slices); the slices of a token split its H.
+inline int combine_slices(int T, int H) {
+  const int vec_per_cta = 256;                     // one float4 per thread per pass
+  const int most = (H / 4 + vec_per_cta - 1) / vec_per_cta;
+  return T >= 1024 ? 1 : (T >= 512 ? std::min(2, most) : std::min(4, most));
+}
 template <typename YT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const YT* __restrict__ Y, const YT* __restrict__ Ys, const float* __restrict__ w,
@@ -39,7 +47,9 @@ combine_kernel(const YT* __restrict__ Y, const YT* __restrict__ Ys, const float*
   }
   __syncthreads();
   const YT* ys = Ys ? Ys + static_cast<size_t>(t) * H : Y + (static_cast<size_t>(T) * k + t) * H;  // shared-expert row
-  for (int v = threadIdx.x; v < H / 4; v += blockDim.x) {
+  // gridDim.y CTAs share the token's row (small micro-batches: more loads in flight); every
+  // element is still summed by one thread in j order, so the result does not depend on it
+  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < H / 4; v += gridDim.y * blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (sizeof(YT) == 4) {
       // fp32 rows: four rows' loads in flight at once, accumulated in j order (measured 15 %
