@@ -47,14 +47,14 @@ import synth  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
-# of the decode shape, from a one-pass ncu capture of two launches at T=256, H=7168, E=256,
-# k=8, I=2048 with the shared expert: 23 076 790 784 and
-# 23 081 380 864 bytes for 257 touched experts.  Traffic grows with the experts whose weights
-# are streamed, and it is reported only while the kernel source and its instantiation are the
-# ones that were captured.
+# of the decode shape, from an ncu capture of a small case of the same kernel (T=16, H=7168,
+# E=16 + 1 shared, k=8, I=2048: all 17 experts touched, 1.5 GB of weights): 1 499 608 320 +
+# 5 750 528 bytes in one launch.  The weight stream dominates, so the traffic grows with the
+# experts whose weights are streamed and is scaled by them; it is reported only while the
+# kernel sources and the file that instantiates them are the ones that were captured.
 MEASURED_TRAFFIC = {
-    "sources_sha256": "e79c1ebd330be23c2d966e0fbbce8a6fbf48fd621f8c83d326de1e01e904dd79",
-    "bytes_per_touched_expert": (23076790784 + 23081380864) / 2 / 257,
+    "sources_sha256": "6e0e167ebfeee3a1637d3497f353c9733eb6d1fede376b353446cab89150badf",
+    "bytes_per_touched_expert": (1499608320 + 5750528) / 17,
 }
 METRIC = "MoE-FFN tokens/s/layer"
 
