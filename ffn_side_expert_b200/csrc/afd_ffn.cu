@@ -92,6 +92,8 @@ struct afd_ffn_handle {
   cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
 
   CUtensorMap tm_w13, tm_w2, tm_wr;
+  CUtensorMap tm_w13i;       // W13 as interleaved gate/up blocks (5-D view) for one-accumulator units
+  bool one = false;          // large W8A8 micro-batches run the one-accumulator GEMMs
   // bf16 large micro-batches: f16 copy of W2 and the f16 activation plane (single-term down GEMM)
   void* w2h = nullptr;       // [E+S][H][I] f16, owned; NULL when unused
   bool act16 = false;
@@ -175,10 +177,31 @@ bool encode_2d(CUtensorMap* m, const void* base, bool byte_elems, uint64_t inner
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false>
+// W13 [G][2I][H] (1- or 2-byte elements) viewed as 5-D {H, 16 rows, gate|up, I/16 blocks, G}, so
+// that one box {128 bytes, 16, 2, 4, 1} holds 64 consecutive gate rows interleaved with their up
+// rows: 16 gate rows, their 16 up rows, the next 16 gate rows, ... (128 rows of 128 bytes, the
+// 128-byte swizzle applied to each row as in a 2-D box).
+bool encode_w13_interleaved(CUtensorMap* m, const void* base, bool byte_elems, uint64_t H, uint64_t I,
+                            uint64_t G) {
+  auto enc = get_encode();
+  if (!enc || I % 64 != 0) return false;
+  const uint64_t esz = byte_elems ? 1 : 2;
+  cuuint64_t dims[5] = {H, 16, 2, I / 16, G};
+  cuuint64_t strides[4] = {H * esz, I * H * esz, 16 * H * esz, 2 * I * H * esz};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / esz), 16, 2, 4, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, byte_elems ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false, bool ONE = false>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<BN, ST, SPLIT, MODE>());
+  return cudaFuncSetAttribute(grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16, ONE>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              gemm_smem_bytes<BN, ST, SPLIT, MODE, ONE>());
 }
 
 // bf16 large micro-batches with f16 activations: gate/up (f16 act plane) and down (f16 operands)
@@ -192,6 +215,17 @@ cudaError_t set_gemm_attr() {
 #define AFD_ACT16_G2_ST 4
 #endif
 constexpr int kAct16BN = 128;
+
+// W8A8 large micro-batches: one-accumulator units of up to kOneBN token rows (GemmShape ONE),
+// kOneST ring stages of 48 KB.  Gate/up units cover 64 act columns, down units 128 output rows.
+// Measured on one B200 machine against the two-accumulator 128-row tiles, A/B in the same call:
+// W8A8 T=8192 4.49-4.54 vs 4.59-4.74 ms per step.  bf16 with f16 activations measured slower
+// this way (T=4096 Zipf: 5.61-5.65 vs 5.16-5.33 ms): its 2-byte token rows, re-read by twice as
+// many units, cost more than the weight re-streams saved, so it keeps the 128-row tiles.
+#ifndef AFD_ONE
+#define AFD_ONE 1
+#endif
+constexpr int kOneBN = 256, kOneST = 4;
 
 // (gate/up, down) kernel pairs of each path and tile shape: N tile and ring stages of each
 // GEMM.  Compile-time tunable for tile sweeps: -DAFD_<path>_BN=.. -DAFD_<path>_ST=..
@@ -325,11 +359,17 @@ cudaError_t set_all_gemm_attrs() {
     e = set_gemm_attr<kAct16BN, AFD_ACT16_G1_ST, false, 0, false, true>();
     if (e != cudaSuccess) return e;
     e = set_gemm_attr<kAct16BN, AFD_ACT16_G2_ST, false, 1, false, true>();
+    if (e != cudaSuccess) return e;
+  }
+  if constexpr (FP8) {
+    e = set_gemm_attr<kOneBN, kOneST, true, 0, false, false, true>();
+    if (e != cudaSuccess) return e;
+    e = set_gemm_attr<kOneBN, kOneST, true, 1, false, false, true>();
   }
   return e;
 }
 
-template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false>
+template <int BN, int ST, bool FP8, int MODE, bool SPLIT, bool ACT16 = false, bool ONE = false>
 void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, cudaStream_t s,
                  const CUtensorMap* a2 = nullptr, const CUtensorMap* b2 = nullptr) {
   if constexpr (MODE == 3) {
@@ -349,8 +389,9 @@ void launch_gemm(int grid, const CUtensorMap& a, const CUtensorMap& b, const Gem
     cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>, a, b, a2 ? *a2 : a,
                        b2 ? *b2 : b, args);
   } else {
-    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16>
-        <<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE>(), s>>>(a, b, a2 ? *a2 : a, b2 ? *b2 : b, args);
+    grouped_gemm_kernel<BN, ST, FP8, MODE, SPLIT, ACT16, ONE>
+        <<<grid, kGemmThreads, gemm_smem_bytes<BN, ST, SPLIT, MODE, ONE>(), s>>>(a, b, a2 ? *a2 : a, b2 ? *b2 : b,
+                                                                             args);
   }
 }
 
@@ -540,10 +581,59 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   launch_gemm<P::bn2, P::st2, FP8, 1, P::split>(grid, h->tm_w2, h->tm_act[shape], g2, s);
 }
 
+// W8A8 large micro-batches on the one-accumulator GEMMs: gate/up units of 64 interleaved act
+// columns, the activation quantisation, then down units of 128 output rows; both with up to
+// kOneBN token rows per unit.
+void run_gemms_one(afd_ffn_handle* h, int T, cudaStream_t s) {
+  const afd_ffn_cfg& c = h->cfg;
+  const int R = T * c.k + T;
+  GemmArgs g1{};
+  g1.single_rows = -1;
+  g1.grp_rows = h->grp_rows;
+  g1.grp_base = h->grp_base;
+  g1.unit_base = h->ub1;
+  g1.G = h->G;
+  g1.K = c.H;
+  g1.a_rows = 2 * c.I;     // scale rows per expert
+  g1.mt_stride = 64;       // act columns per unit
+  g1.second_off = c.I;     // up row = gate row + I
+  g1.out = h->act;         // fp32 SwiGLU rows
+  g1.out_ld = c.I;
+  g1.a_policy = kEvictNormal;
+  g1.a_scale = h->w.w13_scale;
+  g1.b_scale = h->xscale;  // hidden row scales
+  g1.err = h->err;
+  record(h, 5, s);
+  launch_gemm<kOneBN, kOneST, true, 0, false, false, true>(h->num_sms, h->tm_w13i, h->tm_xp[1], g1, s);
+  record(h, 6, s);
+  quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
+  GemmArgs g2 = g1;
+  g2.unit_base = h->ub2;
+  g2.K = c.I;
+  g2.a_rows = c.H;
+  g2.mt_stride = 128;      // output rows per unit
+  g2.second_off = 0;
+  g2.out = h->Y;
+  g2.out_ld = c.H;
+  g2.a_scale = h->w.w2_scale;
+  g2.b_scale = h->ascale;
+  record(h, 7, s);
+  launch_gemm<kOneBN, kOneST, true, 1, false, false, true>(h->num_sms, h->tm_w2, h->tm_act[1], g2, s);
+}
+
 int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   const bool narrow = use_narrow(h, T);
   const int shape = narrow ? kNarrow : kWide;
+  if (!narrow && h->one) {
+    record(h, 4, s);
+    build_schedule_kernel<<<1, 512, 0, s>>>(offsets, c.E, c.n_shared, T, c.k, kOneBN, kOneBN, c.I / 64, c.H / 128,
+                                            h->grp_rows, h->grp_base, h->ub1, h->ub2, h->tile_base, h->tile_done,
+                                            h->err);
+    run_gemms_one(h, T, s);
+    AFD_CUDA(h, cudaGetLastError());
+    return AFD_OK;
+  }
   int bn1, bn2, gate_rows;
   auto pick = [&](auto p) {
     using P = decltype(p);
@@ -780,6 +870,17 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
       // a zero (or NaN) bound still gives every row the scale 1
       h->f16_bound = std::max(2.0f * C / 32768.0f, 1e-30f);
     }
+  }
+  // large W8A8 micro-batches run the one-accumulator GEMMs, whose gate/up side reads W13 through
+  // the interleaved 5-D view
+  if (AFD_ONE && h->fp8 && static_cast<int64_t>(c.T_max) * c.k > 32 * static_cast<int64_t>(c.E)) {
+    if (!encode_w13_interleaved(&h->tm_w13i, weights->w13, h->fp8, c.H, c.I, G)) {
+      if (h->w2h) cudaFree(h->w2h);
+      cudaFree(h->ws);
+      delete h;
+      return AFD_ERR_INVALID_ARG;
+    }
+    h->one = true;
   }
   e = h->fp8 ? set_all_gemm_attrs<true>() : set_all_gemm_attrs<false>();
   if (e != cudaSuccess) { cudaFree(h->ws); if (h->w2h) cudaFree(h->w2h); delete h; return cuda_fail(nullptr, e); }

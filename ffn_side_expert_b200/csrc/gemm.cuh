@@ -89,11 +89,16 @@ struct GemmArgs {
   int mt1;                   // gate/up units per N tile (I / 128)
 };
 
-template <int BN, bool SPLIT_B = false, int MODE = 0>
+// ONE (W8A8 large micro-batches): one 128-row weight tile and one accumulator per unit, with up
+// to BN = 256 token rows -- so a unit still fits twice in TMEM.  Gate/up (MODE 0) then loads the
+// tile interleaved (for each lane quarter 16 gate rows and their 16 up rows, from a 5-D tensor
+// map), and a unit covers 64 act columns; down (MODE 1) covers 128 output rows.  Fewer, wider
+// units: a tail of a few rows rides in a balanced tile instead of costing a unit of its own.
+template <int BN, bool SPLIT_B = false, int MODE = 0, bool ONE = false>
 struct GemmShape {
   static constexpr bool kFused = MODE == 3;
-  static constexpr int kNA = MODE == 2 ? 3 : 2;   // weight tiles per stage
-  static constexpr int kNDU = MODE == 2 ? 1 : 2;  // accumulators per unit
+  static constexpr int kNA = MODE == 2 ? 3 : (ONE ? 1 : 2);     // weight tiles per stage
+  static constexpr int kNDU = (MODE == 2 || ONE) ? 1 : 2;       // accumulators per unit
   static constexpr int kATile = 128 * 128;              // one 128-row x 128-byte weight tile
   static constexpr int kAStage = kNA * kATile;
   static constexpr int kBRows = BN;                     // token rows of a tile
@@ -121,6 +126,7 @@ struct GemmShape {
   static_assert(kColsUsed <= 512, "TMEM has 512 columns");
   static_assert(BN % 16 == 0 && BN <= 256, "N tile");
   static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+  static_assert(!ONE || ((MODE == 0 || MODE == 1) && !SPLIT_B), "one-accumulator units: wide gate/up or down");
 };
 
 // Shared memory: the group schedule (one int4 per group: first unit, rows, first row), then
@@ -128,10 +134,10 @@ struct GemmShape {
 constexpr int kMaxGroups = 257;
 constexpr int kSchedBytes = (kMaxGroups + 1) * 16;
 
-template <int BN, int STAGES, bool SPLIT_B, int MODE = 0>
+template <int BN, int STAGES, bool SPLIT_B, int MODE = 0, bool ONE = false>
 constexpr int gemm_smem_bytes() {
   return (MODE == 3 ? 2 : 1) * kSchedBytes + 1024 /*alignment slack*/ +
-         STAGES * GemmShape<BN, SPLIT_B, MODE>::kStageBytes + 256 /*barriers*/;
+         STAGES * GemmShape<BN, SPLIT_B, MODE, ONE>::kStageBytes + 256 /*barriers*/;
 }
 
 // Largest g with tab[g].x (first unit of group g) <= u; the table sits in shared memory.
@@ -185,8 +191,13 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const int4* tab, 
     const int ntiles = (grows + BN - 1) / BN;
     w.mt = local / ntiles;
     const int nt = local - w.mt * ntiles;
-    w.rows = min(BN, grows - nt * BN);
-    w.row0 = gs.z + nt * BN;
+    // wide tiles: a group's rows are spread evenly over its ntiles tiles (sizes rounded up to 16)
+    // instead of full tiles and a ragged last one -- an expert with 270 rows runs 96 + 96 + 78
+    // rather than 128 + 128 + 14, and a small-N MMA costs nearly as much as a 128-row one.
+    // (ntiles - 1) * sz < grows, since sz <= BN, so the last tile is never empty.
+    const int sz = BN >= 128 ? min(BN, ((grows + ntiles - 1) / ntiles + 15) & ~15) : BN;
+    w.rows = min(sz, grows - nt * sz);
+    w.row0 = gs.z + nt * sz;
     w.split = 0;
     w.kc0 = 0;
     w.kc1 = kchunks;
@@ -230,7 +241,7 @@ __device__ __forceinline__ bool wait_tile(const int* cnt, int need, volatile int
 // f16 operands) -- f16 keeps 10 mantissa bits where bf16 keeps 7, so one term suffices.  Each
 // token row is stored divided by its power-of-two scale b_scale[row] (f16_row_scale: the row's
 // bound on |act| stays inside the f16 range), and the down epilogue multiplies it back.
-template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool ACT16 = false>
+template <int BN, int STAGES, bool FP8, int MODE, bool SPLIT_B, bool ACT16 = false, bool ONE = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -238,7 +249,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   static_assert(!(SPLIT_B && (FP8 || (MODE != 1 && MODE != 3))), "two-term B only for the bf16 down GEMM");
   static_assert(!((MODE == 2 || MODE == 3) && FP8), "router and fused modes run on bf16");
   static_assert(!ACT16 || (!FP8 && !SPLIT_B && (MODE == 0 || MODE == 1)), "f16 activations: wide bf16 GEMMs");
-  using S = GemmShape<BN, SPLIT_B, MODE>;
+  static_assert(!ONE || (FP8 && !ACT16), "one-accumulator units serve the W8A8 wide GEMMs");
+  using S = GemmShape<BN, SPLIT_B, MODE, ONE>;
   constexpr int kNacc = S::kNacc;
   constexpr int kKChunk = FP8 ? 128 : 64;  // elements per 128-byte row slice
 
@@ -341,9 +353,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t fb = full + 8u * s;
         const int x = kc * kKChunk;
         mbar_arrive_expect_tx(full + 8u * s, tx);
-        // the tile pair (MODE 0/1) or the three router planes (MODE 2)
+        if constexpr (ONE && MODE == 0) {
+          // 64 act columns: blocks 4 mt .. 4 mt + 3 of 16 gate rows, each with its up rows
+          tma_load_5d(st, mA, fb, x, 0, 0, 4 * w.mt, w.g, apol);
+        } else {
+          // the tile pair (MODE 0/1), one tile (ONE down) or the three router planes (MODE 2)
 #pragma unroll
-        for (int i = 0; i < S::kNA; ++i) tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
+          for (int i = 0; i < S::kNA; ++i) tma_load_2d(st + i * S::kATile, mA, fb, x, ya + i * soff, apol);
+        }
         const uint32_t sb = st + S::kAStage;
         for (int b = 0; b < nbox; ++b) tma_load_2d(sb + b * boxr * 128, mB, fb, x, brow0 + b * boxr, kEvictLast);
         if (two) {
@@ -394,7 +411,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_mma<false>(d0, da2 + 2 * kk, db + 2 * kk, idesc, 1u);
           } else {
             tc_mma<FP8>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-            tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+            if constexpr (S::kNDU == 2) tc_mma<FP8>(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
             if constexpr (SPLIT_B && !S::kConcat) {  // the lo plane as separate MMAs
               if (down) {
                 const uint64_t dl = sw128_desc(st + S::kAStage + S::kBTile);
@@ -452,6 +469,33 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int n = c + i;
             if (n < w.rows && e < args.a_rows)
               lg[static_cast<size_t>(w.row0 + n) * args.out_ld + e] = __uint_as_float(r0[i]);
+          }
+        }
+      } else if constexpr (ONE && MODE == 0) {
+        // interleaved gate/up: this warp's lane quarter holds act columns jc0 .. jc0 + 15; lane l
+        // reads the gate row of column jc0 + l (l < 16) or the up row of column jc0 + l - 16.
+        // For each 16-token chunk the gate lane takes tokens 0..7 and the up lane tokens 8..15,
+        // trading the other half with its partner lane (l xor 16).
+        const int up = lane >> 4;
+        const int jc = w.mt * args.mt_stride + 16 * q + (lane & 15);  // act column
+        const float sa = __ldg(args.a_scale + static_cast<size_t>(w.g) * args.a_rows + up * args.second_off + jc);
+        for (int c = c_first; c < w.n16; c += kCStep) {
+          float sb_lane = 0.f;  // token scales, lane i < 16 holding token c + i
+          if (lane < 16 && c + lane < w.rows) sb_lane = __ldg(args.b_scale + w.row0 + c + lane);
+          uint32_t r0[16];
+          tmem_ld16(t0 + c, r0);
+          tmem_ld_wait(r0);
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r0[i]) * sa * __shfl_sync(0xffffffffu, sb_lane, i);
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            const float other = __shfl_xor_sync(0xffffffffu, up ? v[n] : v[n + 8], 16);
+            const float g = up ? other : v[n];
+            const float uv = up ? v[n + 8] : other;
+            const int tok = c + n + 8 * up;
+            if (tok < w.rows)  // fp32 SwiGLU row, quantised per row before the down GEMM
+              static_cast<float*>(args.out)[static_cast<size_t>(w.row0 + tok) * args.out_ld + jc] = silu_f(g) * uv;
           }
         }
       } else {
