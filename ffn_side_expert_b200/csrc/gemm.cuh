@@ -472,8 +472,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
       } else if constexpr (ONE && MODE == 0) {
-        // interleaved gate/up: this warp's lane quarter holds act columns jc0 .. jc0 + 15; lane l
-        // reads the gate row of column jc0 + l (l < 16) or the up row of column jc0 + l - 16.
+        // interleaved gate/up: this warp's lane quarter q holds act columns jc0 .. jc0 + 15, with
+        // jc0 = 64 mt + 16 q; lane l reads the gate row of column jc0 + l (l < 16) or the up row of
+        // column jc0 + l - 16.
         // For each 16-token chunk the gate lane takes tokens 0..7 and the up lane tokens 8..15,
         // trading the other half with its partner lane (l xor 16).
         const int up = lane >> 4;
