@@ -63,3 +63,17 @@ def test_clock_summary_keeps_only_the_timed_window(tmp_path):
     c.f, c.first, c.last = f, 6, 6                           # no sample inside a short region
     s2 = c.summary()
     assert s2["samples"] == 1 and s2["sm_mhz"] == 1320.0
+
+
+def test_shape_entry_carries_its_own_measurement():
+    import argparse
+    cfg, acct = _acct("w8a8_8192")
+    r = {"cfg": cfg, "acct": acct, "ms": 4.3, "kernel_ms": 2.3, "stage_ms": np.linspace(0.01, 0.09, 9),
+         "clocks": {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 5}}
+    args = argparse.Namespace(steps=20, warmup=5)
+    e = bench.report_shape(args, 1, r)
+    assert set(e) >= {"value", "unit", "ms_per_step", "dtype", "config", "roofline", "path_roofline",
+                      "stage_ms", "gpu_launches", "clocks"}
+    assert abs(e["value"] - cfg.T / 4.3e-3) < 1.0 and e["dtype"] == "fp8_e4m3"
+    assert e["config"]["workload"] == "w8a8_8192" and e["gpu_launches"] == 10 * 20
+    assert e["roofline"]["bound"] == "tensor" and len(e["stage_ms"]) == 9
