@@ -96,3 +96,31 @@ def test_w8a8_expert_parallel_layer_on_one_rank(name, T):
             ep.close()
         dist.destroy_process_group()
         L.close()
+
+
+def test_expert_parallel_layer_on_the_wide_tiles():
+    # T*k rows per local expert block well above 32 per expert: the rank's expert handle runs the
+    # large-micro-batch GEMMs (f16 activations with their row scales, computed by
+    # afd_ffn_expert_rows for rows that arrive already grouped), and the shared expert too
+    cfg = synth.MoEConfig("epw", T=600, H=256, E=4, k=2, I=256, S=1, seed=33)
+    L = Layer(cfg, redraws=_redraws(cfg))
+    port = 26700 + os.getpid() % 1000
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    ep = None
+    try:
+        d = L.dev
+        ep = ExpertParallelFfn(H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, T_max=cfg.T, router_w=d["router_w"],
+                               local_w13=d["w13"][:cfg.E], local_w2=d["w2"][:cfg.E],
+                               shared_w13=d["w13"][cfg.E], shared_w2=d["w2"][cfg.E])
+        out = ep.forward(L.h)
+        torch.cuda.synchronize()
+        assert afd.afd_ffn_rows_error() == afd.AFD_OK
+        ref = L.oracle()
+        err = rel_max_err(to64(out), ref["out"])
+        print(f"expert-parallel wide T={cfg.T}: max|err|/RMS = {err:.4e} (bar {BF16_TOL})")
+        assert err <= BF16_TOL, err
+    finally:
+        if ep is not None:
+            ep.close()
+        dist.destroy_process_group()
+        L.close()
