@@ -91,8 +91,9 @@ typedef struct afd_ffn_handle afd_ffn_handle;
  * the caller's tensors: the router weights as three bf16 planes (hi + mid + lo = Wr to ~2^-27),
  * and -- for bf16 weights when T_max * k > 32 * E, i.e. when large micro-batches are possible --
  * an f16 copy of W2 ([E+n_shared][H][I], exact for |w| in [2^-14, 65504]; if a weight exceeds
- * 65504 no copy is kept and the two-term bf16 down GEMM is used).  *out receives the handle
- * (NULL on failure).  Synchronous. */
+ * 65504 no copy is kept and the two-term bf16 down GEMM is used) together with one pass over W13
+ * for the bound max ||wg_i|| ||wu_i|| that sizes the f16 activations' per-row power-of-two
+ * scales.  *out receives the handle (NULL on failure).  Synchronous. */
 int afd_ffn_create(const afd_ffn_cfg *cfg, const afd_ffn_weights *weights, afd_ffn_handle **out);
 
 /* Free the workspace and the handle (after synchronising the device).  NULL is a no-op. */
