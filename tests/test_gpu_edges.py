@@ -253,10 +253,13 @@ def test_w8a8_zero_rows():
 
 def test_wide_bf16_without_the_f16_copy_of_w2():
     # a W2 weight beyond the f16 range (1e5) leaves the handle without its f16 copy of W2, so the
-    # large-micro-batch path runs the two-term bf16 down GEMM (hi and lo act planes) instead
+    # large-micro-batch path runs the two-term bf16 down GEMM (hi and lo act planes) instead.
+    # The weight sits in an act column that is exactly zero (its gate row is zero, silu(0) = 0),
+    # so the outputs keep their usual range and the 2e-2 x RMS bar stays meaningful.
     cfg = synth.MoEConfig("wide", T=600, H=256, E=2, k=1, I=256, S=1, seed=24)
 
     def big_weight(ex):
+        ex["w13"][1, 3] = 0
         ex["w2"][1, 7, 3] = 1.0e5
 
     L = Layer(cfg, redraws=_redraws(cfg), edit_experts=big_weight)
