@@ -7,8 +7,9 @@ One step = one afd_ffn_forward over one micro-batch (router, top-k, dispatch, ga
 with SwiGLU, down GEMM, shared expert, combine).  Default workload: the DeepSeek-V3 shaped
 decode micro-batch (T=256, H=7168, E=256 + 1 shared, top-8, I=2048, bf16) on seeded
 synthetic inputs.  On one GPU the same line also carries, under "shapes", the T=4096
-Zipf-skewed bf16 micro-batch and the T=8192 W8A8 chunk, each timed the same way (K steps
-after W warm-ups) with its own roofline, stage split and clock record.  Its 22.6 GB of expert weights are far larger than the 126 MB L2, so no
+Zipf-skewed bf16 micro-batch, the T=8192 W8A8 chunk and the T=256 W8A8 decode micro-batch,
+each timed the same way (K steps after W warm-ups) with its own roofline, stage split and
+clock record.  Its 22.6 GB of expert weights are far larger than the 126 MB L2, so no
 flush is needed between steps.  N > 1 runs one independent replica per GPU (the layer is
 not sharded: no collective on the data path); value = total tokens of all ranks / the
 slowest rank's time.  --impl reference times the fp64 CPU oracle on a bounded sample of the
@@ -756,7 +757,7 @@ def main(argv=None):
                     help="profiling only: override the micro-batch size (a smaller case of the same kernels)")
     ap.add_argument("--E", type=int, default=None,
                     help="profiling only: override the number of routed experts")
-    ap.add_argument("--shapes", default="dsv3_4096,w8a8_8192",
+    ap.add_argument("--shapes", default="dsv3_4096,w8a8_8192,w8a8_256",
                     help="comma-separated workloads timed after the headline one (1 GPU only; '' for none)")
     ap.add_argument("--period", action="store_true",
                     help="measure the FFN-service micro-pipeline period with a host attention stub (1 GPU)")
