@@ -61,6 +61,8 @@ _L = ctypes.c_int64
 _SIGNATURES = {
     "afd_ffn_create": (ctypes.c_int, [ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(afd_ffn_weights),
                                       ctypes.POINTER(ctypes.c_void_p)]),
+    "afd_ffn_create_ex": (ctypes.c_int, [ctypes.POINTER(afd_ffn_cfg), ctypes.POINTER(afd_ffn_weights),
+                                         ctypes.c_uint32, ctypes.POINTER(ctypes.c_void_p)]),
     "afd_ffn_destroy": (None, [_P]),
     "afd_ffn_route": (ctypes.c_int, [_P, _P, _I, _P, _P, _P]),
     "afd_ffn_permute": (ctypes.c_int, [_P, _P, _P, _I, _P, _P, _P, _P, _P]),
@@ -157,6 +159,17 @@ def afd_ffn_create(cfg: afd_ffn_cfg, weights: afd_ffn_weights):
     h = ctypes.c_void_p()
     st = _lib.afd_ffn_create(ctypes.byref(cfg) if cfg is not None else None,
                              ctypes.byref(weights) if weights is not None else None, ctypes.byref(h))
+    return st, (h.value if st == AFD_OK else None)
+
+
+AFD_CREATE_NO_W2_COPY = 1
+
+
+def afd_ffn_create_ex(cfg: afd_ffn_cfg, weights: afd_ffn_weights, flags: int):
+    """Returns (status, handle or None)."""
+    h = ctypes.c_void_p()
+    st = _lib.afd_ffn_create_ex(ctypes.byref(cfg) if cfg is not None else None,
+                                ctypes.byref(weights) if weights is not None else None, flags, ctypes.byref(h))
     return st, (h.value if st == AFD_OK else None)
 
 
@@ -363,7 +376,7 @@ class AfdFfn:
     w2_scale [E+S,H] fp32.  The tensors are referenced for the handle's lifetime.
     """
 
-    def __init__(self, *, T_max, H, E, k, I, n_shared, fp8, weights):
+    def __init__(self, *, T_max, H, E, k, I, n_shared, fp8, weights, flags=0):
         dt = AFD_DT_FP8_E4M3 if fp8 else AFD_DT_BF16
         self.cfg = afd_ffn_cfg(T_max, H, E, k, I, n_shared, dt, dt,
                                1 if weights.get("router_bias") is not None else 0)
@@ -371,9 +384,9 @@ class AfdFfn:
         w = afd_ffn_weights(_ptr(weights["router_w"]), _ptr(weights.get("router_bias")),
                             _ptr(weights["w13"]), _ptr(weights["w2"]),
                             _ptr(weights.get("w13_scale")), _ptr(weights.get("w2_scale")))
-        st, self.h = afd_ffn_create(self.cfg, w)
+        st, self.h = afd_ffn_create_ex(self.cfg, w, flags)
         if st != AFD_OK:
-            raise AfdError(st, "afd_ffn_create")
+            raise AfdError(st, "afd_ffn_create_ex")
         self._events = None
 
     def close(self):

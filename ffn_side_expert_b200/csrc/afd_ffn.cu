@@ -738,9 +738,15 @@ int afd_ffn_get_info(const afd_ffn_handle* h, afd_ffn_cfg* cfg, int32_t* device)
 }
 
 int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_ffn_handle** out) {
+  return afd_ffn_create_ex(cfg, weights, 0u, out);
+}
+
+int afd_ffn_create_ex(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, uint32_t flags,
+                      afd_ffn_handle** out) {
   if (!out) return AFD_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg || !weights) return AFD_ERR_INVALID_ARG;
+  if (flags & ~static_cast<uint32_t>(AFD_CREATE_NO_W2_COPY)) return AFD_ERR_INVALID_ARG;
   int st = validate_cfg(cfg);
   if (st != AFD_OK) return st;
   if ((st = validate_weights(cfg, weights)) != AFD_OK) return st;
@@ -838,7 +844,8 @@ int afd_ffn_create(const afd_ffn_cfg* cfg, const afd_ffn_weights* weights, afd_f
   if (!ok) { cudaFree(h->ws); delete h; return AFD_ERR_INVALID_ARG; }
   // bf16 handles that can see large micro-batches keep an f16 copy of W2 for the single-term
   // down GEMM (unless a weight exceeds the f16 range; then the two-term bf16 path stays)
-  if (AFD_ACT16 && !h->fp8 && static_cast<int64_t>(c.T_max) * c.k > 32 * static_cast<int64_t>(c.E)) {
+  if (AFD_ACT16 && !h->fp8 && !(flags & AFD_CREATE_NO_W2_COPY) &&
+      static_cast<int64_t>(c.T_max) * c.k > 32 * static_cast<int64_t>(c.E)) {
     const size_t n = G * c.H * static_cast<size_t>(c.I);
     e = cudaMalloc(&h->w2h, n * 2);
     if (e != cudaSuccess) { cudaFree(h->ws); delete h; return cuda_fail(nullptr, e); }

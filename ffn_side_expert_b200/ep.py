@@ -228,6 +228,8 @@ class ExpertParallelFfn:
     them raise PeerLost -- a rank that arrives after another gave up finds "abort" and raises
     too, instead of entering a collective alone.  A rank that has left, or a store that can no
     longer be reached, is reported as PeerLost before this rank launches any exchange.
+    The aborted step stays decided, so a layer that raised PeerLost does not continue: the
+    caller rebuilds the group (and the layer) without the lost rank.
     Without a store, a short process-group timeout is the bound.
     """
 

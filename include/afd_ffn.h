@@ -96,6 +96,14 @@ typedef struct afd_ffn_handle afd_ffn_handle;
  * scales.  *out receives the handle (NULL on failure).  Synchronous. */
 int afd_ffn_create(const afd_ffn_cfg *cfg, const afd_ffn_weights *weights, afd_ffn_handle **out);
 
+/* afd_ffn_create with options.  flags: 0, or AFD_CREATE_NO_W2_COPY -- keep no f16 copy of W2
+ * (saves (E+n_shared)*H*I*2 bytes of device memory, 7.5 GB at H=7168, I=2048, E=256+1; large
+ * bf16 micro-batches then run the two-term bf16 down GEMM, which multiplies two activation
+ * planes and is slower).  Other bits: AFD_ERR_INVALID_ARG. */
+#define AFD_CREATE_NO_W2_COPY 1u
+int afd_ffn_create_ex(const afd_ffn_cfg *cfg, const afd_ffn_weights *weights, uint32_t flags,
+                      afd_ffn_handle **out);
+
 /* Free the workspace and the handle (after synchronising the device).  NULL is a no-op. */
 void afd_ffn_destroy(afd_ffn_handle *h);
 

@@ -52,6 +52,8 @@ def test_create_rejects_bad_config_on_host(kw, status):
 
 
 def test_create_rejects_bad_weights_on_host():
+    st, _ = afd.afd_ffn_create_ex(_cfg(), _W, 2)            # unknown option bit, refused on the host
+    assert st == afd.AFD_ERR_INVALID_ARG
     st, _ = afd.afd_ffn_create(_cfg(), afd.afd_ffn_weights(None, None, 512, 768, None, None))
     assert st == afd.AFD_ERR_INVALID_ARG
     st, _ = afd.afd_ffn_create(_cfg(), afd.afd_ffn_weights(257, None, 512, 768, None, None))
@@ -122,7 +124,7 @@ def test_bounded_wait_check_needs_a_device():
 
 
 def _declared_params(header=afd.HEADER_PATH):
-    """name -> list of parameter kinds ('ptr', 'i32', 'i64', 'f32') from include/afd_ffn.h."""
+    """name -> list of parameter kinds ('ptr', 'i32', 'u32', 'i64', 'f32') from include/afd_ffn.h."""
     import re
     with open(header) as f:
         text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
@@ -137,6 +139,8 @@ def _declared_params(header=afd.HEADER_PATH):
                 kinds.append("i64")
             elif "float" in p:
                 kinds.append("f32")
+            elif "uint32_t" in p:
+                kinds.append("u32")
             else:
                 assert re.search(r"\b(int32_t|int)\b", p), p
                 kinds.append("i32")
@@ -147,7 +151,8 @@ def _declared_params(header=afd.HEADER_PATH):
 def _kind(ct):
     if ct in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(ct, type(ctypes.POINTER(ctypes.c_int))):
         return "ptr"
-    return {ctypes.c_int32: "i32", ctypes.c_int: "i32", ctypes.c_int64: "i64", ctypes.c_float: "f32"}[ct]
+    return {ctypes.c_int32: "i32", ctypes.c_int: "i32", ctypes.c_uint32: "u32", ctypes.c_int64: "i64",
+            ctypes.c_float: "f32"}[ct]
 
 
 def _declared_arities(header=afd.HEADER_PATH):

@@ -268,3 +268,35 @@ def test_wide_bf16_without_the_f16_copy_of_w2():
         _check_layer(L, cfg.T)
     finally:
         L.close()
+
+
+def test_no_w2_copy_option():
+    # AFD_CREATE_NO_W2_COPY: a bf16 handle for large micro-batches keeps no f16 copy of W2 (device
+    # memory drops by (E+S) H I 2 bytes) and its wide path runs the two-term bf16 down GEMM
+    cfg = synth.MoEConfig("wide_big", T=300, H=2048, E=2, k=1, I=8192, S=1, seed=34)   # a 100 MB copy
+    L = Layer(cfg, redraws=_redraws(cfg))
+    try:
+        copy_bytes = (cfg.E + cfg.S) * cfg.H * cfg.I * 2
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        lean = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S, fp8=False,
+                          weights=L.dev, flags=afd.AFD_CREATE_NO_W2_COPY)
+        free1 = torch.cuda.mem_get_info()[0]
+        full = afd.AfdFfn(T_max=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.S, fp8=False,
+                          weights=L.dev)
+        free2 = torch.cuda.mem_get_info()[0]
+        assert (free1 - free2) - (free0 - free1) >= copy_bytes - (4 << 20)   # the copy, within pages
+        outs = []
+        for mod in (lean, full):
+            out = torch.empty_like(L.h)
+            mod.forward(L.h, out)
+            torch.cuda.synchronize()
+            assert mod.get_error() == 0
+            outs.append(out)
+        ref = L.oracle()
+        for out in outs:
+            assert rel_max_err(to64(out), ref["out"]) <= BF16_TOL
+        lean.close()
+        full.close()
+    finally:
+        L.close()
