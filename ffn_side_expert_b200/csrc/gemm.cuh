@@ -11,7 +11,9 @@
 // streams full 128-row weight tiles.  A work unit is two 128-row weight tiles (gate rows j..,
 // up rows I+j.. for MODE 0; down rows h.., h+128.. for MODE 1) against one tile of up to BN
 // token rows, accumulated over K into two fp32 TMEM accumulators; SwiGLU (MODE 0) and the
-// scales of the W8A8 path are applied in the epilogue straight from TMEM.
+// scales of the W8A8 path are applied in the epilogue straight from TMEM.  W8A8 large
+// micro-batches use one-accumulator units instead (GemmShape ONE: one interleaved gate/up tile
+// against up to 256 token rows).
 //
 // bf16 path, two-term activations: the gate/up epilogue stores the fp32 SwiGLU output as
 // hi = bf16(act) and lo = bf16(act - hi) in two planes, and the down GEMM (SPLIT_B) multiplies
@@ -24,14 +26,17 @@
 // its gate/up units first, then its down units.  A gate/up epilogue publishes each finished act
 // tile with a release increment of its (expert, N tile) counter; the producer of a down unit
 // waits (acquire, bounded) until all I/128 act tiles of its rows are in, then issues its loads.
-// Every dependency lies earlier in each CTA's unit order, so the waits always end; the HBM-bound
-// weight stream of late gate/up units overlaps the tensor-heavier down units.
+// Every dependency lies earlier in each CTA's unit order and the launch is cooperative (every
+// CTA resident at once), so the waits always end; the HBM-bound weight stream of late gate/up
+// units overlaps the tensor-heavier down units.
 //
 // MODE 2 (router): the fp32 router weights are stored once as three bf16 planes hi + mid + lo
 // (each the bf16 rounding of what the previous planes leave), so Wr is represented to ~2^-27
 // relative; bf16 x bf16 products are exact in fp32 and the three planes accumulate into one
-// TMEM accumulator.  The reduction over H can be split across units (partial logits, summed
-// in order by the top-k kernel) to spread a small micro-batch over more SMs.
+// TMEM accumulator.  The reduction over H is split across units (partial logits, summed in
+// order in fp32 by the top-k kernel): into stretches of at most 1024 elements, which keeps the
+// tensor core's accumulation error far below the gate-weight tolerance, and further to spread a
+// small micro-batch over more SMs.
 //
 // Pipeline: one ring of STAGES shared-memory stages, each holding the weight tiles and the
 // token tile of one 128-byte K chunk.  Warp roles (64 + 32 x kEpiWarps threads): warp 0 lane 0
