@@ -270,6 +270,10 @@ def time_forward(layer, h, out, cfg, args, world, local_rank) -> dict:
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # torch creates an event's CUDA handle at its first record; create every handle now, so that
+    # inside the timed region the stream carries only the two records around the dominant kernel
+    for e in [x for pair in kev for x in pair] + [t_start, t_end]:
+        e.record(stream)
 
     barrier(world)
     torch.cuda.synchronize()
