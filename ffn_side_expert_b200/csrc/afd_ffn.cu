@@ -471,7 +471,7 @@ int run_route(afd_ffn_handle* h, const void* hidden, int T, int32_t* idx, float*
   record(h, 1, s);
   // selection and gate weights from the summed partial logits, a warp per token
   const float* bias = c.has_router_bias ? h->w.router_bias : nullptr;
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(h->part, ksplit, bias, T, c.E, c.k, idx, w);
+  launch_router_topk(h->part, ksplit, bias, T, c.E, c.k, idx, w, s);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
 }
@@ -1132,7 +1132,7 @@ extern "C" int afd_ffn_route_static(const void* hidden, const float* router_w, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok, nsplit);
   router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(hidden), router_w, part, T, H, E, per);
-  router_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, router_bias, T, E, k, topk_idx, topk_w);
+  launch_router_topk(part, nsplit, router_bias, T, E, k, topk_idx, topk_w, s);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;

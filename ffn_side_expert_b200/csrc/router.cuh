@@ -90,29 +90,50 @@ router_logits_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __re
   }
 }
 
-// One warp per token.  part: [nsplit][T][E] partial logits (summed in split order); bias: [E]
-// or nullptr.  Writes the k selected experts (descending logit, ties to the lower index) and
-// the softmax of their logits.
+// WPT warps per token (one, or four when the partial logits come in many splits: a small
+// micro-batch's router GEMM splits H widely to fill the SMs).  part: [nsplit][T][E] partial
+// logits; warp g of a token adds splits g*per .. (g+1)*per - 1 in order, then warp 0 adds the
+// WPT sums in order (a fixed order, independent of scheduling); bias: [E] or nullptr.  Writes
+// the k selected experts (descending logit, ties to the lower index) and the softmax of their
+// logits.  blockDim = 256: 8 / WPT tokens per CTA.
+template <int WPT>
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __restrict__ bias,
                    int T, int E, int k, int32_t* __restrict__ idx, float* __restrict__ w) {
+  __shared__ float red[WPT > 1 ? 8 * 8 * 32 : 1];  // [token in CTA][warp of the token][i][lane]
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+  const int warp = threadIdx.x >> 5;
+  const int tl = warp / WPT, g = warp % WPT;
+  const int t = blockIdx.x * (8 / WPT) + tl;
   float v[8];
   unsigned taken = 0;
-  // partial logits summed in split order; the eight loads of one split are independent, so a
-  // lane waits for one memory round trip per split rather than one per (split, value)
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) {
-    const float* ps = part + (static_cast<size_t>(sp) * T + t) * E;
+  if (t < T) {
+    // the eight loads of one split are independent, so a lane waits for one memory round trip
+    // per split rather than one per (split, value)
+    const int per = (nsplit + WPT - 1) / WPT;
+    const int s1 = min(nsplit, (g + 1) * per);
+    for (int sp = g * per; sp < s1; ++sp) {
+      const float* ps = part + (static_cast<size_t>(sp) * T + t) * E;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) v[i] += ps[e];
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) v[i] += ps[e];
+      }
     }
   }
+  if constexpr (WPT > 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[((tl * WPT + g) * 8 + i) * 32 + lane] = v[i];
+    __syncthreads();
+    if (g != 0) return;
+    for (int gg = 1; gg < WPT; ++gg) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += red[((tl * WPT + gg) * 8 + i) * 32 + lane];
+    }
+  }
+  if (t >= T) return;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
@@ -151,6 +172,16 @@ router_topk_kernel(const float* __restrict__ part, int nsplit, const float* __re
     idx[static_cast<size_t>(t) * k + lane] = my_e;
     w[static_cast<size_t>(t) * k + lane] = z / sum;
   }
+}
+
+// Selection and gate weights from nsplit partial logits: four warps per token when the partials
+// come in eight or more splits (a small micro-batch), else one.
+inline void launch_router_topk(const float* part, int nsplit, const float* bias, int T, int E, int k, int32_t* idx,
+                               float* w, cudaStream_t s) {
+  if (nsplit >= 8)
+    router_topk_kernel<4><<<(T + 1) / 2, 256, 0, s>>>(part, nsplit, bias, T, E, k, idx, w);
+  else
+    router_topk_kernel<1><<<(T + 7) / 8, 256, 0, s>>>(part, nsplit, bias, T, E, k, idx, w);
 }
 
 // Router weights for the tensor-core router: Wr (fp32) -> three bf16 planes [3][n] with
