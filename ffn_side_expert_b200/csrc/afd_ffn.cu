@@ -666,14 +666,13 @@ int run_expert_gemm(afd_ffn_handle* h, const int32_t* offsets, int T, cudaStream
 int run_combine(afd_ffn_handle* h, const float* w, const int32_t* pos, int T, void* out, cudaStream_t s) {
   const afd_ffn_cfg& c = h->cfg;
   record(h, 8, s);
-  const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(combine_slices(T, c.H)));
-  if (h->fp8)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->Y), nullptr, w, pos, T,
-                                                       c.k, c.H, T * c.k, c.n_shared, static_cast<__nv_bfloat16*>(out),
-                                                       h->err);
+  if (h->fp8)  // H is a multiple of 256
+    combine8_kernel<<<dim3(static_cast<unsigned>(T), static_cast<unsigned>(combine8_slices(T, c.H))), kCombine8Threads,
+                      0, s>>>(reinterpret_cast<const __nv_bfloat16*>(h->Y), nullptr, w, pos, T, c.k, c.H, T * c.k,
+                              c.n_shared, static_cast<__nv_bfloat16*>(out), h->err);
   else
-    combine_kernel<float><<<grid, 256, 0, s>>>(h->Y, nullptr, w, pos, T, c.k, c.H, T * c.k, c.n_shared,
-                                               static_cast<__nv_bfloat16*>(out), h->err);
+    combine_kernel<float><<<dim3(static_cast<unsigned>(T), static_cast<unsigned>(combine_slices(T, c.H))), 256, 0, s>>>(
+        h->Y, nullptr, w, pos, T, c.k, c.H, T * c.k, c.n_shared, static_cast<__nv_bfloat16*>(out), h->err);
   record(h, 9, s);
   AFD_CUDA(h, cudaGetLastError());
   return AFD_OK;
@@ -1254,10 +1253,14 @@ extern "C" int afd_ffn_combine_rows_bf16(const void* Y, const void* Ys, const fl
   int st = rows_err_word(&err);
   if (st != AFD_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  combine_kernel<__nv_bfloat16><<<dim3(static_cast<unsigned>(T), static_cast<unsigned>(combine_slices(T, H))), 256, 0,
-                                  s>>>(static_cast<const __nv_bfloat16*>(Y),
-                                                  static_cast<const __nv_bfloat16*>(Ys), topk_w, pos, T, k, H, T * k,
-                                                  Ys ? 1 : 0, static_cast<__nv_bfloat16*>(out), err);
+  if (H % 8 == 0)
+    combine8_kernel<<<dim3(static_cast<unsigned>(T), static_cast<unsigned>(combine8_slices(T, H))), kCombine8Threads, 0,
+                      s>>>(static_cast<const __nv_bfloat16*>(Y), static_cast<const __nv_bfloat16*>(Ys), topk_w, pos, T,
+                           k, H, T * k, Ys ? 1 : 0, static_cast<__nv_bfloat16*>(out), err);
+  else
+    combine_kernel<__nv_bfloat16><<<dim3(static_cast<unsigned>(T), static_cast<unsigned>(combine_slices(T, H))), 256, 0,
+                                    s>>>(static_cast<const __nv_bfloat16*>(Y), static_cast<const __nv_bfloat16*>(Ys),
+                                         topk_w, pos, T, k, H, T * k, Ys ? 1 : 0, static_cast<__nv_bfloat16*>(out), err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(nullptr, e);
   return AFD_OK;
