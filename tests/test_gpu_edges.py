@@ -300,3 +300,46 @@ def test_no_w2_copy_option():
         full.close()
     finally:
         L.close()
+
+
+def test_w8a8_row_codes_bit_exact():
+    # R9 on the device: every dispatched row's e4m3 codes and fp32 scale equal the oracle's bit for
+    # bit (the codes are integer decisions taken in fp32 on both sides).  Rows 0..63 put an exact
+    # e4m3 tie in every element: the row maximum is 448 * 2^j, so the scale is 2^j and x / s is
+    # exact, and the other values are midpoints between neighbouring e4m3 values (ties to even)
+    # at every binade; the rest are N(0, 1) rows, with one all-zero row (scale 1).
+    from oracle import fp8 as ofp8
+    T, H, E, k = 512, 1024, 16, 4
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    grid = np.array(sorted({float(ofp8.e4m3_round(np.float64(v))) for v in np.linspace(0.001, 448, 4000)}))
+    mids = (grid[:-1] + grid[1:]) / 2
+    for t in range(64):
+        j = t % 16 - 8
+        row = rng.choice(mids, size=H) * np.where(rng.random(H) < 0.5, -1.0, 1.0)
+        row[0] = 448.0
+        x[t] = (row * 2.0 ** j).astype(np.float32)
+    x[100] = 0.0
+    hidden32 = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(hidden32.float()[:64], torch.from_numpy(x[:64]))  # the ties survive bf16
+    idx = torch.from_numpy(np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32))
+    dev = "cuda"
+    hidden, idx_d = hidden32.to(dev), idx.to(dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    rows = torch.empty((T * k + T, H), dtype=torch.uint8, device=dev)
+    scales = torch.empty(T * k + T, dtype=torch.float32, device=dev)
+    scratch = torch.empty(2 * ((T + 127) // 128) * E, dtype=torch.int32, device=dev)
+    st = afd.afd_ffn_dispatch_rows_fp8(hidden, idx_d, T, k, E, H, 1, counts, offsets, pos, src, rows, scales, scratch)
+    assert st == afd.AFD_OK
+    assert afd.afd_ffn_rows_error() == afd.AFD_OK
+    q, s = ofp8.quantize_rows(hidden32.float().numpy())
+    codes = ofp8.e4m3_encode(q)
+    src_h = src.cpu().numpy().astype(np.int64)
+    tok = np.concatenate([src_h, np.arange(T)])            # routed rows, then every token once
+    got_codes, got_scales = rows.cpu().numpy(), scales.cpu().numpy()
+    assert np.array_equal(got_scales.view(np.uint32), s[tok].view(np.uint32))
+    bad = np.argwhere(got_codes != codes[tok])
+    assert bad.size == 0, f"{len(bad)} codes differ, first at row {bad[0][0]} column {bad[0][1]}"
