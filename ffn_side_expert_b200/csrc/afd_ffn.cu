@@ -566,7 +566,7 @@ void run_gemms(afd_ffn_handle* h, int T, cudaStream_t s) {
   launch_gemm<P::bn1, P::st1, FP8, 0, false>(grid, h->tm_w13, h->tm_xp[shape], g1, s);
   record(h, 6, s);
   if (FP8)
-    quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
+    quantize_act_kernel<<<(R + 1) / 2, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
   GemmArgs g2 = g1;
   g2.unit_base = h->ub2;
   g2.K = c.I;
@@ -606,7 +606,7 @@ void run_gemms_one(afd_ffn_handle* h, int T, cudaStream_t s) {
   record(h, 5, s);
   launch_gemm<kOneBN, kOneST, true, 0, false, false, true>(h->num_sms, h->tm_w13i, h->tm_xp[1], g1, s);
   record(h, 6, s);
-  quantize_act_kernel<<<(R + 7) / 8, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
+  quantize_act_kernel<<<(R + 1) / 2, 256, 0, s>>>(static_cast<const float*>(h->act), R, c.I, h->actq, h->ascale);
   GemmArgs g2 = g1;
   g2.unit_base = h->ub2;
   g2.K = c.I;
