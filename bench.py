@@ -49,13 +49,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the fused bf16 expert kernel
 # of the decode shape, from an ncu capture of a small case of the same kernel (T=16, H=7168,
-# E=16 + 1 shared, k=8, I=2048: all 17 experts touched, 1.5 GB of weights): 1 499 610 112 +
-# 5 076 480 bytes in one launch.  The weight stream dominates, so the traffic grows with the
+# E=16 + 1 shared, k=8, I=2048: all 17 experts touched, 1.5 GB of weights): 1 499 667 712 +
+# 5 541 888 bytes in one launch.  The weight stream dominates, so the traffic grows with the
 # experts whose weights are streamed and is scaled by them; it is reported only while the
 # kernel sources and the file that instantiates them are the ones that were captured.
 MEASURED_TRAFFIC = {
-    "sources_sha256": "6f0773fffaeb61ea349cf273818b0e24d476cefe98ab430bff4bd655365c15e7",
-    "bytes_per_touched_expert": (1499610112 + 5076480) / 17,
+    "sources_sha256": "bf25b6660b8e09b8d7390c6d39413cbf5b1ccdef277ed8ffb4afae47bae4a6b6",
+    "bytes_per_touched_expert": (1499667712 + 5541888) / 17,
 }
 METRIC = "MoE-FFN tokens/s/layer"
 
